@@ -1,0 +1,1100 @@
+// Strided indexer top-k for B200 (sm_100a).
+//
+// Operation (vLLM PR #42169 report, "实现拆解"; SGLang PR #34167 code
+// excerpt): for each row r of fp32 logits at logits + r*row_stride, the k
+// largest of the first L_r values, as row-local indices ordered by value
+// descending and index ascending, padded with -1 past min(k, L_r).
+//
+// Design (one HBM pass, no global scratch):
+//   * One producer warp streams a row (or a chunk of it) into a ring of
+//     shared-memory stages with cp.async.bulk (TMA bulk copies, no
+//     multicast) completing on mbarriers.
+//   * Sixteen consumer warps turn each fp32 into an order-preserving uint32
+//     key only when it can still matter: a running threshold T (the exact
+//     k-th largest key among the entries seen so far) filters the stream, and
+//     survivors are appended to a shared-memory candidate buffer in index
+//     order. Because tiles arrive in index order, a later entry equal to T
+//     always loses its tie, so the filter is "key > T".
+//   * When the buffer would overflow, a radix select (adaptive 8-bit windows
+//     over the key range actually present) finds the exact k-th key, and a
+//     stable compaction keeps the k winners, ties by lowest index. This is
+//     the pages' histogram / run_cumsum / threshold / gt-eq split, made exact
+//     and deterministic.
+//   * At the end a stable LSD radix sort orders the <= k winners and the
+//     output row is written with -1 padding.
+//   * Many rows: one CTA per row, persistent over rows; the producer runs
+//     ahead into the next row while consumers finish the current one.
+//   * Few long rows: a thread-block cluster splits a row into contiguous
+//     chunks. Ranks merge through distributed shared memory: a cluster-wide
+//     histogram over the candidates narrows the threshold, ranks publish
+//     counts, and each rank writes its survivors into the leader's shared
+//     memory at rank-ordered offsets (so index order, hence the tie rule, is
+//     preserved). Cluster barriers separate the phases; every CTA reaches
+//     every barrier.
+//
+// Coding rules taken from the SGLang PR #34167 discussion: a distributed
+// shared-memory address is only ever a 32-bit shared::cluster address used
+// with ld/st.shared::cluster, never merged with a CTA-local pointer; k is a
+// runtime value; kernel attributes are set per kernel per device.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "dsa_topk.h"
+
+#define DSA_EXPORT extern "C" __attribute__((visibility("default")))
+
+namespace dsa {
+
+constexpr int kNumConsumerWarps = 16;
+constexpr int kConsumerThreads = kNumConsumerWarps * 32;       // 512
+constexpr int kThreads = kConsumerThreads + 32;                // + producer warp
+constexpr int kStageElems = 4096;                              // 16 KB per stage
+constexpr uint32_t kStageBytes = kStageElems * 4;
+constexpr int kStages = 8;                                     // 128 KB ring
+constexpr int kMaxK = DSA_TOPK_MAX_K;
+constexpr int kCap = kMaxK + 2 * kStageElems;                  // candidate buffer entries
+constexpr int kGatherOff = kMaxK;                              // cluster gather region
+constexpr int kGatherCap = kCap - kGatherOff;
+constexpr int kSortCountOff = 2 * kMaxK;                       // sort counters alias free space
+constexpr int kMaxEntriesPerThread = (kCap + kConsumerThreads - 1) / kConsumerThreads;
+constexpr uint32_t kNanKey = 0xFFC00000u;  // key of the canonical quiet NaN
+constexpr unsigned kFull = 0xFFFFFFFFu;
+constexpr unsigned long long kWaitLimitNs = 500000000ull;     // 0.5 s per pipeline wait
+constexpr int kMaxRadixRounds = 4;  // 32-bit keys, >= 8 bits resolved per round
+
+// Sticky status bits (g_status).
+constexpr unsigned kStatusWaitTimeout = 1u;   // a pipeline wait gave up
+constexpr unsigned kStatusSelectBroken = 2u;  // a radix round lost its invariant
+
+static_assert(kSortCountOff + kNumConsumerWarps * 256 <= kCap, "sort counters must fit");
+static_assert(kGatherCap >= kMaxK, "gather region must hold k entries");
+static_assert(kCap - kMaxK >= kStageElems, "a stage must fit after a compaction");
+
+enum Mode : int { kAcceptAll = 0, kFilter = 1, kRejectAll = 2 };
+
+struct __align__(128) Smem {
+  float ring[kStages][kStageElems];
+  uint32_t ckey[kCap];
+  uint32_t cidx[kCap];
+  uint32_t hist[256];
+  uint32_t phist[2][256];  // published to the cluster
+  uint32_t ghist[256];
+  uint32_t wtot[2][kNumConsumerWarps];
+  uint32_t red[6][kNumConsumerWarps];
+  uint32_t pub[8];  // published to the cluster
+  uint32_t bc[8];
+  uint32_t skip[4];
+  unsigned long long full[kStages];
+  unsigned long long empty[kStages];
+};
+static_assert(sizeof(Smem) <= 232448, "shared memory budget (227 KB)");
+
+__device__ unsigned int g_status;  // sticky status bits, see kStatus*
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait: returns false (and records the status bit) after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_status, kStatusWaitTimeout);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void bar_consumers() {
+  asm volatile("bar.sync 1, %0;" ::"r"(kConsumerThreads) : "memory");
+}
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_index() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::
+          : "memory");
+}
+// Address of the same shared variable in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t dsmem_map(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ uint32_t dsmem_ld(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void dsmem_st(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// ------------------------------------------------------------- key mapping
+// Order-preserving map fp32 -> uint32: larger key = larger value; every NaN
+// maps to the key of +qNaN (above +inf); -0.0 maps to +0.0's key.
+__device__ __forceinline__ uint32_t to_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (x != x) u = 0x7fc00000u;
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+// Inverse of to_key for non-NaN keys.
+__device__ __forceinline__ float from_key(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+// ------------------------------------------------------------ row geometry
+// A work item is the slice [c0, c1) of one row. Its bytes are fetched as the
+// 16-byte aligned span that covers them; entries outside [c0, c1) are masked.
+struct Span {
+  const char* src;   // 16-byte aligned start
+  int64_t j0;        // row-local index of the first float of the span
+  uint64_t bytes;    // span length, multiple of 16
+  int nst;           // stages
+};
+
+__device__ __forceinline__ Span make_span(const float* row, int64_t c0, int64_t c1) {
+  Span sp;
+  if (c1 <= c0) {
+    sp.src = reinterpret_cast<const char*>(row);
+    sp.j0 = c0;
+    sp.bytes = 0;
+    sp.nst = 0;
+    return sp;
+  }
+  const uintptr_t a = reinterpret_cast<uintptr_t>(row + c0);
+  const uintptr_t e = reinterpret_cast<uintptr_t>(row + c1);
+  const uintptr_t as = a & ~static_cast<uintptr_t>(15);
+  const uintptr_t ee = (e + 15) & ~static_cast<uintptr_t>(15);
+  sp.src = reinterpret_cast<const char*>(as);
+  sp.j0 = c0 - static_cast<int64_t>((a - as) >> 2);
+  sp.bytes = ee - as;
+  sp.nst = static_cast<int>((sp.bytes + kStageBytes - 1) / kStageBytes);
+  return sp;
+}
+
+__device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+__device__ __forceinline__ int64_t clamp_len(const int32_t* lengths, int64_t row, int64_t row_stride) {
+  int64_t L = lengths[row];
+  if (L < 0) L = 0;
+  if (L > row_stride) L = row_stride;
+  return L;
+}
+
+// Producer: issue every stage of one work item into the ring.
+__device__ __forceinline__ void produce_item(Smem& s, const Span& sp, int& stage, uint32_t& phase) {
+  for (int t = 0; t < sp.nst; ++t) {
+    mbar_wait(&s.empty[stage], phase ^ 1u);
+    const uint64_t off = static_cast<uint64_t>(t) * kStageBytes;
+    const uint64_t rem = sp.bytes - off;
+    const uint32_t bytes = rem < kStageBytes ? static_cast<uint32_t>(rem) : kStageBytes;
+    mbar_arrive_expect_tx(&s.full[stage], bytes);
+    bulk_g2s(&s.ring[stage][0], sp.src + off, bytes, &s.full[stage]);
+    if (++stage == kStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+}
+
+// ------------------------------------------------------ block-level helpers
+struct MinMax {
+  uint32_t mn, mx;
+};
+
+// min / max key over entries [base, base+n) (all consumer threads).
+__device__ MinMax block_minmax(Smem& s, int base, int n, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+  for (int e = tid; e < n; e += kConsumerThreads) {
+    const uint32_t key = s.ckey[base + e];
+    mn = min(mn, key);
+    mx = max(mx, key);
+  }
+  mn = __reduce_min_sync(kFull, mn);
+  mx = __reduce_max_sync(kFull, mx);
+  if (lane == 0) {
+    s.red[0][w] = mn;
+    s.red[1][w] = mx;
+  }
+  bar_consumers();
+  const uint32_t a = lane < kNumConsumerWarps ? s.red[0][lane] : 0xFFFFFFFFu;
+  const uint32_t b = lane < kNumConsumerWarps ? s.red[1][lane] : 0u;
+  MinMax r;
+  r.mn = __reduce_min_sync(kFull, a);
+  r.mx = __reduce_max_sync(kFull, b);
+  bar_consumers();  // red[0..1] may be rewritten by the next call
+  return r;
+}
+
+// Bucket search over a 256-bin histogram in descending digit order: finds b
+// with (#keys in bins > b) < need <= (#keys in bins >= b). Warp 0 writes
+// bc[0] = b, bc[1] = #keys in bins > b. Caller synchronises.
+__device__ __forceinline__ void find_bucket_warp0(const uint32_t* hist, uint32_t need, uint32_t* bc, int lane) {
+  uint32_t c[8], sum = 0;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    c[t] = hist[255 - 8 * lane - t];
+    sum += c[t];
+  }
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const uint32_t excl = incl - sum;
+  if (excl < need && need <= incl) {
+    uint32_t acc = excl;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (acc + c[t] >= need) {
+        bc[0] = 255u - 8u * lane - t;
+        bc[1] = acc;
+        break;
+      }
+      acc += c[t];
+    }
+  }
+}
+
+// Narrow [lo, hi] to bucket b of the window starting at bit sh.
+__device__ __forceinline__ void narrow(uint32_t& lo, uint32_t& hi, int sh, uint32_t b) {
+  const uint32_t keep_hi = (sh + 8 >= 32) ? 0u : ~((1u << (sh + 8)) - 1u);
+  const uint32_t blo = (lo & keep_hi) | (b << sh);
+  const uint32_t bhi = blo | ((1u << sh) - 1u);
+  lo = max(lo, blo);
+  hi = min(hi, bhi);
+}
+
+// Window for the next radix step: 8 bits ending at the highest differing bit.
+__device__ __forceinline__ int window_shift(uint32_t lo, uint32_t hi) {
+  const int h = 31 - __clz(lo ^ hi);
+  return h >= 7 ? h - 7 : 0;
+}
+
+// Histogram of keys in [lo, hi] over entries [base, base+n) into hist[256]
+// (already zeroed). Lanes with the same digit combine into one atomic.
+__device__ __forceinline__ void histogram(const Smem& s, uint32_t* hist, int base, int n, uint32_t lo, uint32_t hi,
+                                          int sh, int tid) {
+  const int lane = tid & 31;
+  const int iters = (n + kConsumerThreads - 1) / kConsumerThreads;
+  for (int it = 0; it < iters; ++it) {
+    const int e = it * kConsumerThreads + tid;
+    uint32_t d = 0xFFFFFFFFu;
+    if (e < n) {
+      const uint32_t key = s.ckey[base + e];
+      if (key >= lo && key <= hi) d = (key >> sh) & 255u;
+    }
+    const uint32_t peers = __match_any_sync(kFull, d);
+    if (d != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[d], static_cast<uint32_t>(__popc(peers)));
+  }
+}
+
+// Stable selection of entries [base, base+n): keep key > T, plus the first
+// need_eq entries with key == T (buffer order = index order). Kept entries go,
+// in order, to dst positions 0.. . Local mode compacts in place at `base`;
+// remote mode stores to the shared::cluster addresses rkey/ridx (+4*(off+pos)).
+template <bool kRemote>
+__device__ void stable_keep(Smem& s, int base, int n, uint32_t T, uint32_t need_eq, uint32_t rkey, uint32_t ridx,
+                            uint32_t off, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  const int per_warp = ((n + kConsumerThreads - 1) / kConsumerThreads) * 32;
+  const int E = per_warp >> 5;
+  const int wbeg = w * per_warp;
+  uint32_t kk[kMaxEntriesPerThread], ii[kMaxEntriesPerThread];
+  uint32_t ngt = 0, neq = 0;
+#pragma unroll
+  for (int it = 0; it < kMaxEntriesPerThread; ++it) {
+    if (it < E) {
+      const int e = wbeg + it * 32 + lane;
+      const bool v = e < n;
+      kk[it] = v ? s.ckey[base + e] : 0u;  // key 0 never occurs: below any T
+      ii[it] = v ? s.cidx[base + e] : 0u;
+      ngt += __popc(__ballot_sync(kFull, kk[it] > T));
+      neq += __popc(__ballot_sync(kFull, kk[it] == T));
+    }
+  }
+  if (lane == 0) {
+    s.red[2][w] = ngt;
+    s.red[3][w] = neq;
+  }
+  bar_consumers();
+  const uint32_t a = lane < kNumConsumerWarps ? s.red[2][lane] : 0u;
+  const uint32_t b = lane < kNumConsumerWarps ? s.red[3][lane] : 0u;
+  uint32_t gt_before = __reduce_add_sync(kFull, lane < w ? a : 0u);
+  uint32_t eq_before = __reduce_add_sync(kFull, lane < w ? b : 0u);
+  const uint32_t lt = lanemask_lt();
+#pragma unroll
+  for (int it = 0; it < kMaxEntriesPerThread; ++it) {
+    if (it < E) {
+      const bool g = kk[it] > T, q = kk[it] == T;
+      const uint32_t gb = __ballot_sync(kFull, g), eb = __ballot_sync(kFull, q);
+      const uint32_t my_gt = gt_before + __popc(gb & lt);
+      const uint32_t my_eq = eq_before + __popc(eb & lt);
+      if (g || (q && my_eq < need_eq)) {
+        const uint32_t pos = my_gt + min(my_eq, need_eq);
+        if (kRemote) {
+          dsmem_st(rkey + 4u * (off + pos), kk[it]);
+          dsmem_st(ridx + 4u * (off + pos), ii[it]);
+        } else {
+          s.ckey[base + pos] = kk[it];
+          s.cidx[base + pos] = ii[it];
+        }
+      }
+      gt_before += __popc(gb);
+      eq_before += __popc(eb);
+    }
+  }
+  bar_consumers();
+}
+
+// Counts of keys > T and == T over entries [0, n) (block-wide, consumers).
+__device__ void count_gt_eq(Smem& s, int n, uint32_t T, uint32_t& ngt, uint32_t& neq, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  uint32_t g = 0, q = 0;
+  for (int e = tid; e < n; e += kConsumerThreads) {
+    const uint32_t key = s.ckey[e];
+    g += key > T;
+    q += key == T;
+  }
+  g = __reduce_add_sync(kFull, g);
+  q = __reduce_add_sync(kFull, q);
+  if (lane == 0) {
+    s.red[4][w] = g;
+    s.red[5][w] = q;
+  }
+  bar_consumers();
+  ngt = __reduce_add_sync(kFull, lane < kNumConsumerWarps ? s.red[4][lane] : 0u);
+  neq = __reduce_add_sync(kFull, lane < kNumConsumerWarps ? s.red[5][lane] : 0u);
+  bar_consumers();
+}
+
+// Exact selection: entries [base, base+n), n > k. Keeps the k largest keys in
+// place, in index order, ties to the lowest index. Returns the k-th largest key.
+__device__ uint32_t select_topk(Smem& s, int base, int n, int k, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  const MinMax r = block_minmax(s, base, n, tid);
+  uint32_t lo = r.mn, hi = r.mx, need = static_cast<uint32_t>(k);
+  for (int round = 0; lo != hi; ++round) {
+    if (round == kMaxRadixRounds) {  // unreachable for a consistent histogram
+      if (tid == 0) atomicOr(&g_status, kStatusSelectBroken);
+      break;
+    }
+    const int sh = window_shift(lo, hi);
+    if (tid < 256) s.hist[tid] = 0u;
+    if (tid == 0) s.bc[0] = 0xFFFFFFFFu;
+    bar_consumers();
+    histogram(s, s.hist, base, n, lo, hi, sh, tid);
+    bar_consumers();
+    if (w == 0) find_bucket_warp0(s.hist, need, s.bc, lane);
+    bar_consumers();
+    if (s.bc[0] == 0xFFFFFFFFu) {  // no bucket holds the need-th key
+      if (tid == 0) atomicOr(&g_status, kStatusSelectBroken);
+      bar_consumers();
+      break;
+    }
+    const uint32_t b = s.bc[0], above_b = s.bc[1];
+    need -= above_b;
+    narrow(lo, hi, sh, b);
+    bar_consumers();  // bc / hist reused by the next round
+  }
+  stable_keep<false>(s, base, n, lo, need, 0u, 0u, 0u, tid);
+  return lo;
+}
+
+// Stable LSD radix sort of entries [src, src+m) (m <= kMaxK) by key
+// descending, using [alt, alt+m) as the other buffer. Ties keep buffer order.
+// Returns the base that holds the sorted entries.
+__device__ int sort_desc(Smem& s, int src, int alt, int m, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  uint32_t* wcnt = s.ckey + kSortCountOff;  // [warp][256]
+  if (tid < 4) s.skip[tid] = 0u;
+  const uint32_t lt = lanemask_lt();
+  for (int pass = 0; pass < 4; ++pass) {
+    const int sh = pass * 8;
+    for (int i = tid; i < kNumConsumerWarps * 256; i += kConsumerThreads) wcnt[i] = 0u;
+    bar_consumers();
+    uint32_t dig[4], lp[4];
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int item = w * 128 + it * 32 + lane;
+      const bool v = item < m;
+      const uint32_t d = v ? ((~s.ckey[src + item]) >> sh) & 255u : 0xFFFFFFFFu;
+      const uint32_t peers = __match_any_sync(kFull, d);
+      const uint32_t c = v ? wcnt[w * 256 + d] : 0u;
+      __syncwarp();
+      if (v && lane == __ffs(peers) - 1) wcnt[w * 256 + d] = c + __popc(peers);
+      __syncwarp();
+      dig[it] = d;
+      lp[it] = c + __popc(peers & lt);
+    }
+    bar_consumers();
+    uint32_t tot = 0, incl = 0;
+    if (tid < 256) {
+      for (int ww = 0; ww < kNumConsumerWarps; ++ww) {
+        const uint32_t c = wcnt[ww * 256 + tid];
+        wcnt[ww * 256 + tid] = tot;
+        tot += c;
+      }
+      if (tot == static_cast<uint32_t>(m)) s.skip[pass] = 1u;
+      incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (lane == 31) s.red[4][w] = incl;
+    }
+    bar_consumers();
+    if (tid < 256) {
+      uint32_t dbase = incl - tot;
+      for (int ww = 0; ww < w; ++ww) dbase += s.red[4][ww];
+      for (int ww = 0; ww < kNumConsumerWarps; ++ww) wcnt[ww * 256 + tid] += dbase;
+    }
+    bar_consumers();
+    if (s.skip[pass]) continue;  // every entry has the same digit: order unchanged
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int item = w * 128 + it * 32 + lane;
+      if (item < m) {
+        const uint32_t dst = wcnt[w * 256 + dig[it]] + lp[it];
+        s.ckey[alt + dst] = s.ckey[src + item];
+        s.cidx[alt + dst] = s.cidx[src + item];
+      }
+    }
+    bar_consumers();
+    const int t = src;
+    src = alt;
+    alt = t;
+  }
+  return src;
+}
+
+__device__ __forceinline__ void write_row(const Smem& s, int R, int m, int k, int32_t* out_row, int tid) {
+  for (int j = tid; j < k; j += kConsumerThreads)
+    out_row[j] = j < m ? static_cast<int32_t>(s.cidx[R + j]) : -1;
+}
+
+// ------------------------------------------------------------ stream phase
+struct StreamState {
+  uint32_t count;  // candidates held (uniform across consumers)
+  int mode;
+  float thr;       // from_key(T) when mode == kFilter
+  int par;         // wtot double-buffer parity
+};
+
+__device__ __forceinline__ void set_threshold(StreamState& st, uint32_t T) {
+  if (T == kNanKey) {
+    st.mode = kRejectAll;
+  } else {
+    st.mode = kFilter;
+    st.thr = from_key(T);
+  }
+}
+
+// Consume one stage: filter, append survivors in index order.
+__device__ __forceinline__ void consume_stage(Smem& s, StreamState& st, int stage, int64_t jbase, int64_t c0,
+                                              int64_t c1, int k, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  const float* src = &s.ring[stage][0];
+  const int o0 = w * 256 + lane * 4, o1 = o0 + 128;
+  const float4 v0 = *reinterpret_cast<const float4*>(src + o0);
+  const float4 v1 = *reinterpret_cast<const float4*>(src + o1);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&s.empty[stage]);  // data is in registers: release the slot
+
+  int64_t lo64 = c0 - jbase, hi64 = c1 - jbase;
+  const int lo = static_cast<int>(lo64 < 0 ? 0 : (lo64 > kStageElems ? kStageElems : lo64));
+  const int hi = static_cast<int>(hi64 < 0 ? 0 : (hi64 > kStageElems ? kStageElems : hi64));
+  const float x0[4] = {v0.x, v0.y, v0.z, v0.w};
+  const float x1[4] = {v1.x, v1.y, v1.z, v1.w};
+  uint32_t f0 = 0, f1 = 0;
+  if (st.mode != kRejectAll) {
+    const bool all = st.mode == kAcceptAll;
+    const float thr = st.thr;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const bool in0 = (o0 + c >= lo) && (o0 + c < hi);
+      const bool in1 = (o1 + c >= lo) && (o1 + c < hi);
+      const bool p0 = all || !(x0[c] <= thr);  // NaN passes any finite threshold
+      const bool p1 = all || !(x1[c] <= thr);
+      f0 |= static_cast<uint32_t>(in0 && p0) << c;
+      f1 |= static_cast<uint32_t>(in1 && p1) << c;
+    }
+  }
+  uint32_t b0[4], b1[4];
+  uint32_t t0 = 0, t1 = 0;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    b0[c] = __ballot_sync(kFull, (f0 >> c) & 1u);
+    b1[c] = __ballot_sync(kFull, (f1 >> c) & 1u);
+    t0 += __popc(b0[c]);
+    t1 += __popc(b1[c]);
+  }
+  if (lane == 0) s.wtot[st.par][w] = t0 + t1;
+  bar_consumers();
+  const uint32_t v = lane < kNumConsumerWarps ? s.wtot[st.par][lane] : 0u;
+  const uint32_t pre = __reduce_add_sync(kFull, lane < w ? v : 0u);
+  const uint32_t tot = __reduce_add_sync(kFull, v);
+  st.par ^= 1;
+  if (tot == 0) return;
+  if (st.count + tot > static_cast<uint32_t>(kCap)) {
+    // Make room. Survivors of this stage passed the old threshold; appending
+    // them after the compaction keeps the buffer a superset of the winners.
+    const uint32_t T = select_topk(s, 0, static_cast<int>(st.count), k, tid);
+    st.count = static_cast<uint32_t>(k);
+    set_threshold(st, T);
+  }
+  if (t0 + t1) {
+    const uint32_t lt = lanemask_lt();
+    uint32_t p0 = st.count + pre, p1 = st.count + pre + t0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      p0 += __popc(b0[c] & lt);
+      p1 += __popc(b1[c] & lt);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if ((f0 >> c) & 1u) {
+        s.ckey[p0] = to_key(x0[c]);
+        s.cidx[p0] = static_cast<uint32_t>(jbase + o0 + c);
+        ++p0;
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if ((f1 >> c) & 1u) {
+        s.ckey[p1] = to_key(x1[c]);
+        s.cidx[p1] = static_cast<uint32_t>(jbase + o1 + c);
+        ++p1;
+      }
+    }
+  }
+  st.count += tot;
+}
+
+// Stream one work item; on return the buffer holds min(k, #valid) winners of
+// the item in index order (exactly the item's top-k when it had >= k entries).
+__device__ __forceinline__ uint32_t stream_item(Smem& s, const Span& sp, int64_t c0, int64_t c1, int k, int& stage,
+                                                uint32_t& phase, int& par, int tid) {
+  StreamState st;
+  st.count = 0;
+  st.mode = kAcceptAll;
+  st.thr = 0.f;
+  st.par = par;
+  for (int t = 0; t < sp.nst; ++t) {
+    mbar_wait(&s.full[stage], phase);
+    consume_stage(s, st, stage, sp.j0 + static_cast<int64_t>(t) * kStageElems, c0, c1, k, tid);
+    if (++stage == kStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+  bar_consumers();  // the last stage's appends land before anyone reads the buffer
+  if (st.count > static_cast<uint32_t>(k)) {
+    select_topk(s, 0, static_cast<int>(st.count), k, tid);
+    st.count = static_cast<uint32_t>(k);
+  }
+  par = st.par;
+  return st.count;
+}
+
+__device__ __forceinline__ void init_pipeline(Smem& s) {
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], kNumConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+}
+
+// --------------------------------------------------------------- kernels
+// Many rows: one CTA per row, persistent over rows (row = blockIdx.x + i*gridDim.x).
+__global__ void __launch_bounds__(kThreads, 1)
+    topk_rows_kernel(const float* __restrict__ logits, int64_t row_stride, const int32_t* __restrict__ lengths,
+                     int64_t num_rows, int k, int32_t* __restrict__ out) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>(smem_raw);
+  init_pipeline(s);
+  const int tid = threadIdx.x;
+  if (tid >= kConsumerThreads) {  // producer warp
+    if (tid == kConsumerThreads) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int64_t row = blockIdx.x; row < num_rows; row += gridDim.x) {
+        const int64_t L = clamp_len(lengths, row, row_stride);
+        produce_item(s, make_span(logits + row * row_stride, 0, L), stage, phase);
+      }
+    }
+    return;
+  }
+  int stage = 0, par = 0;
+  uint32_t phase = 0;
+  for (int64_t row = blockIdx.x; row < num_rows; row += gridDim.x) {
+    const int64_t L = clamp_len(lengths, row, row_stride);
+    const Span sp = make_span(logits + row * row_stride, 0, L);
+    const uint32_t m = stream_item(s, sp, 0, L, k, stage, phase, par, tid);
+    const int R = m ? sort_desc(s, 0, kMaxK, static_cast<int>(m), tid) : 0;
+    write_row(s, R, static_cast<int>(m), k, out + row * static_cast<int64_t>(k), tid);
+    bar_consumers();  // outputs read cidx before the next row appends
+  }
+}
+
+// Few long rows: a cluster of CTAs per row (grid = num_rows * cluster size).
+__global__ void __launch_bounds__(kThreads, 1)
+    topk_cluster_kernel(const float* __restrict__ logits, int64_t row_stride, const int32_t* __restrict__ lengths,
+                        int64_t num_rows, int k, int32_t* __restrict__ out) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>(smem_raw);
+  init_pipeline(s);
+  const int tid = threadIdx.x;
+  const uint32_t rank = cluster_rank();
+  const uint32_t ncta = cluster_size();
+  const int64_t row = cluster_index();
+  // every CTA of the cluster takes the same branch (row is per cluster)
+  if (row >= num_rows) return;
+  const int64_t L = clamp_len(lengths, row, row_stride);
+  int64_t chunk = (L + ncta - 1) / ncta;
+  chunk = (chunk + 3) & ~static_cast<int64_t>(3);
+  const int64_t c0 = min64(L, static_cast<int64_t>(rank) * chunk);
+  const int64_t c1 = min64(L, c0 + chunk);
+  const float* row_ptr = logits + row * row_stride;
+  const Span sp = make_span(row_ptr, c0, c1);
+  if (tid >= kConsumerThreads) {  // producer warp: issue, then leave the cluster barriers to consumers
+    if (tid == kConsumerThreads) {
+      int stage = 0;
+      uint32_t phase = 0;
+      produce_item(s, sp, stage, phase);
+    }
+    return;
+  }
+  const int w = tid >> 5, lane = tid & 31;
+  int stage = 0, par = 0;
+  uint32_t phase = 0;
+  const uint32_t m = static_cast<uint32_t>(min64(k, L));
+  if (m == 0) {  // L == 0 for every rank alike: nothing streamed, no merge
+    if (rank == 0) write_row(s, 0, 0, k, out + row * static_cast<int64_t>(k), tid);
+    return;
+  }
+  const uint32_t n_r = stream_item(s, sp, c0, c1, k, stage, phase, par, tid);
+
+  // ---- merge phase 1: publish (count, min key, max key) of this rank
+  const MinMax mm = block_minmax(s, 0, static_cast<int>(n_r), tid);
+  if (tid == 0) {
+    s.pub[0] = n_r;
+    s.pub[1] = mm.mn;
+    s.pub[2] = mm.mx;
+  }
+  cluster_barrier();
+  if (w == 0) {
+    uint32_t n = 0, mn = 0xFFFFFFFFu, mx = 0u;
+    if (lane < static_cast<int>(ncta)) {
+      const uint32_t a = dsmem_map(smem_addr(&s.pub[0]), lane);
+      n = dsmem_ld(a);
+      mn = dsmem_ld(a + 4);
+      mx = dsmem_ld(a + 8);
+    }
+    const bool full_rank = lane < static_cast<int>(ncta) && n == static_cast<uint32_t>(k);
+    const uint32_t N = __reduce_add_sync(kFull, n);
+    const uint32_t gmin = __reduce_min_sync(kFull, mn);
+    const uint32_t gmax = __reduce_max_sync(kFull, mx);
+    // a rank holding k entries >= its min bounds the global k-th key from below
+    const uint32_t B = __reduce_max_sync(kFull, full_rank ? mn : 0u);
+    const bool any_full = __ballot_sync(kFull, full_rank) != 0;
+    if (lane == 0) {
+      s.bc[2] = N;
+      s.bc[3] = any_full ? B : gmin;
+      s.bc[4] = gmax;
+      s.bc[5] = gmin;
+    }
+  }
+  bar_consumers();
+  const uint32_t N = s.bc[2];
+  uint32_t lo = s.bc[3], hi = s.bc[4];
+  const uint32_t gmin = s.bc[5];
+  bar_consumers();
+  uint32_t need = m, S = N;
+  bool exact = false;
+  if (N <= static_cast<uint32_t>(kGatherCap)) {
+    lo = gmin;  // everything fits at the leader
+  } else {
+    // ---- merge phase 2: cluster-wide histogram rounds until the survivors fit
+    int hp = 0;
+    for (int round = 0;; ++round) {
+      if (lo == hi || round == kMaxRadixRounds + 1) {
+        if (lo != hi && tid == 0) atomicOr(&g_status, kStatusSelectBroken);
+        exact = true;
+        break;
+      }
+      const int sh = window_shift(lo, hi);
+      if (tid < 256) s.phist[hp][tid] = 0u;
+      if (tid == 0) s.bc[0] = 0xFFFFFFFFu;
+      bar_consumers();
+      histogram(s, s.phist[hp], 0, static_cast<int>(n_r), lo, hi, sh, tid);
+      cluster_barrier();
+      if (tid < 256) {
+        const uint32_t a = smem_addr(&s.phist[hp][tid]);
+        uint32_t g = 0;
+        for (uint32_t r = 0; r < ncta; ++r) g += dsmem_ld(dsmem_map(a, r));
+        s.ghist[tid] = g;
+      }
+      bar_consumers();
+      if (w == 0) find_bucket_warp0(s.ghist, need, s.bc, lane);
+      bar_consumers();
+      if (s.bc[0] == 0xFFFFFFFFu) {  // identical on every rank: the same sums
+        if (tid == 0) atomicOr(&g_status, kStatusSelectBroken);
+        exact = true;
+        lo = hi;
+        bar_consumers();
+        break;
+      }
+      const uint32_t b = s.bc[0], above_b = s.bc[1];
+      need -= above_b;
+      S = (m - need) + s.ghist[b];  // keys above the bucket + keys in it
+      narrow(lo, hi, sh, b);
+      bar_consumers();
+      hp ^= 1;
+      if (S <= static_cast<uint32_t>(kGatherCap)) break;
+    }
+  }
+  // ---- merge phase 3: publish this rank's survivor counts
+  // exact: keep key > T plus a rank-ordered share of key == T; else keep key >= lo
+  const uint32_t T = exact ? lo : lo - 1u;
+  uint32_t g_r, q_r;
+  count_gt_eq(s, static_cast<int>(n_r), T, g_r, q_r, tid);
+  if (tid == 0) {
+    s.pub[4] = g_r;
+    s.pub[5] = exact ? q_r : 0u;
+  }
+  cluster_barrier();
+  if (w == 0) {
+    uint32_t g = 0, q = 0;
+    if (lane < static_cast<int>(ncta)) {
+      const uint32_t a = dsmem_map(smem_addr(&s.pub[4]), lane);
+      g = dsmem_ld(a);
+      q = dsmem_ld(a + 4);
+    }
+    // ranks hold contiguous, increasing index ranges: rank order is index order
+    uint32_t q_incl = q;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(kFull, q_incl, o);
+      if (lane >= o) q_incl += v;
+    }
+    const uint32_t q_excl = q_incl - q;
+    const uint32_t keep_q = exact ? (need > q_excl ? min(q, need - q_excl) : 0u) : 0u;
+    const uint32_t cnt = g + keep_q;
+    uint32_t c_incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(kFull, c_incl, o);
+      if (lane >= o) c_incl += v;
+    }
+    if (lane == static_cast<int>(rank)) {
+      s.bc[6] = c_incl - cnt;  // my offset at the leader
+      s.bc[7] = keep_q;
+    }
+    const uint32_t total = __shfl_sync(kFull, c_incl, 31);
+    if (lane == 0) s.bc[2] = total;
+  }
+  bar_consumers();
+  const uint32_t my_off = s.bc[6], my_keep = s.bc[7], total = s.bc[2];
+  // ---- merge phase 4: copy survivors, in index order, into the leader
+  const uint32_t rkey = dsmem_map(smem_addr(&s.ckey[kGatherOff]), 0);
+  const uint32_t ridx = dsmem_map(smem_addr(&s.cidx[kGatherOff]), 0);
+  stable_keep<true>(s, 0, static_cast<int>(n_r), T, exact ? my_keep : 0u, rkey, ridx, my_off, tid);
+  cluster_barrier();
+  if (rank != 0) return;
+  // ---- leader: exact top-m of the gathered survivors, sort, write
+  if (total > m) select_topk(s, kGatherOff, static_cast<int>(total), static_cast<int>(m), tid);
+  const int R = sort_desc(s, kGatherOff, 0, static_cast<int>(m), tid);
+  write_row(s, R, static_cast<int>(m), k, out + row * static_cast<int64_t>(k), tid);
+}
+
+// ------------------------------------------------------------------ host
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0, minor = 0;
+  int max_cluster = 0;  // largest supported cluster (16 or 8), 0 if none
+  bool ready = false;
+};
+
+constexpr int kMaxDevices = 64;
+static DeviceInfo g_dev[kMaxDevices];
+static std::mutex g_dev_mu;
+
+static int device_setup(int dev, DeviceInfo* out) {
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    cudaDeviceProp p;
+    if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return DSA_ERR_NO_DEVICE;
+    if (p.major != 10) return DSA_ERR_NO_DEVICE;
+    d.sms = p.multiProcessorCount;
+    d.major = p.major;
+    d.minor = p.minor;
+    const int smem = static_cast<int>(sizeof(Smem));
+    if (cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess) {
+      cudaGetLastError();
+      return DSA_ERR_CONFIG;
+    }
+    d.max_cluster = 0;
+    for (int cs : {16, 8}) {
+      if (cs > 8 &&
+          cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+              cudaSuccess) {
+        cudaGetLastError();
+        continue;
+      }
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = cs;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(cs, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int nclusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&nclusters, topk_cluster_kernel, &cfg) == cudaSuccess && nclusters > 0) {
+        d.max_cluster = cs;
+        break;
+      }
+      cudaGetLastError();
+    }
+    d.ready = true;
+  }
+  *out = d;
+  return DSA_OK;
+}
+
+// Launch plan from host-known sizes only.
+static void plan(const DeviceInfo& d, int64_t num_rows, int64_t row_stride, int* cs_out, int64_t* grid_out) {
+  constexpr int64_t kMinChunk = 16384;  // elements per rank worth a cluster merge
+  int cs = 1;
+  if (num_rows < d.sms && d.max_cluster > 1) {
+    int64_t want = d.sms / (num_rows > 0 ? num_rows : 1);
+    while (cs * 2 <= want && cs * 2 <= d.max_cluster && row_stride / (cs * 2) >= kMinChunk) cs *= 2;
+  }
+  *cs_out = cs;
+  if (cs == 1)
+    *grid_out = num_rows < d.sms ? num_rows : d.sms;
+  else
+    *grid_out = num_rows * cs;
+}
+
+static int check_args(const void* logits, int64_t row_stride, const void* lengths, int64_t num_rows, int32_t k,
+                      const void* out) {
+  if (k < 1 || k > kMaxK) return DSA_ERR_BAD_K;
+  if (row_stride < 1) return DSA_ERR_BAD_STRIDE;
+  if (num_rows < 0) return DSA_ERR_BAD_ROWS;
+  if (num_rows > 0 && row_stride > INT64_MAX / num_rows) return DSA_ERR_OVERFLOW;
+  if (num_rows > 0 && num_rows > INT64_MAX / k) return DSA_ERR_OVERFLOW;
+  if (num_rows == 0) return DSA_OK;
+  if (!logits || !lengths || !out) return DSA_ERR_NULL_POINTER;
+  if ((reinterpret_cast<uintptr_t>(logits) | reinterpret_cast<uintptr_t>(lengths) |
+       reinterpret_cast<uintptr_t>(out)) &
+      3u)
+    return DSA_ERR_MISALIGNED;
+  return DSA_OK;
+}
+
+static int current_device(DeviceInfo* info) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return DSA_ERR_NO_DEVICE;
+  }
+  return device_setup(dev, info);
+}
+
+static int launch(const DeviceInfo& d, const float* logits, int64_t row_stride, const int32_t* lengths,
+                  int64_t num_rows, int32_t k, int32_t* out, cudaStream_t stream) {
+  int cs;
+  int64_t grid;
+  plan(d, num_rows, row_stride, &cs, &grid);
+  if (grid > 0x7fffffff) return DSA_ERR_OVERFLOW;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = sizeof(Smem);
+  cfg.stream = stream;
+  cudaError_t e;
+  if (cs == 1) {
+    e = cudaLaunchKernelEx(&cfg, topk_rows_kernel, logits, row_stride, lengths, num_rows, static_cast<int>(k), out);
+  } else {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, logits, row_stride, lengths, num_rows, static_cast<int>(k),
+                           out);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return DSA_ERR_LAUNCH;
+  }
+  return DSA_OK;
+}
+
+}  // namespace dsa
+
+DSA_EXPORT int dsa_topk(const float* logits, int64_t row_stride, const int32_t* lengths, int64_t num_rows,
+                        int32_t k, int32_t* out_idx, dsa_stream_t stream) {
+  int rc = dsa::check_args(logits, row_stride, lengths, num_rows, k, out_idx);
+  if (rc != DSA_OK || num_rows == 0) return rc;
+  dsa::DeviceInfo d;
+  rc = dsa::current_device(&d);
+  if (rc != DSA_OK) return rc;
+  return dsa::launch(d, logits, row_stride, lengths, num_rows, k, out_idx, stream);
+}
+
+DSA_EXPORT int dsa_topk_host(const float* h_logits, int64_t row_stride, const int32_t* h_lengths, int64_t num_rows,
+                             int32_t k, int32_t* h_out, float* d_logits, int32_t* d_lengths, int32_t* d_out,
+                             dsa_stream_t stream) {
+  int rc = dsa::check_args(h_logits, row_stride, h_lengths, num_rows, k, h_out);
+  if (rc != DSA_OK || num_rows == 0) return rc;
+  rc = dsa::check_args(d_logits, row_stride, d_lengths, num_rows, k, d_out);
+  if (rc != DSA_OK) return rc;
+  dsa::DeviceInfo d;
+  rc = dsa::current_device(&d);
+  if (rc != DSA_OK) return rc;
+  const size_t in_bytes = static_cast<size_t>(num_rows) * static_cast<size_t>(row_stride) * sizeof(float);
+  if (cudaMemcpyAsync(d_logits, h_logits, in_bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(d_lengths, h_lengths, static_cast<size_t>(num_rows) * sizeof(int32_t),
+                      cudaMemcpyHostToDevice, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return DSA_ERR_LAUNCH;
+  }
+  rc = dsa::launch(d, d_logits, row_stride, d_lengths, num_rows, k, d_out, stream);
+  if (rc != DSA_OK) return rc;
+  if (cudaMemcpyAsync(h_out, d_out, static_cast<size_t>(num_rows) * k * sizeof(int32_t), cudaMemcpyDeviceToHost,
+                      stream) != cudaSuccess) {
+    cudaGetLastError();
+    return DSA_ERR_LAUNCH;
+  }
+  return DSA_OK;
+}
+
+DSA_EXPORT int dsa_topk_plan(int64_t num_rows, int64_t row_stride, int32_t k, int32_t* cluster_size, int32_t* grid) {
+  if (k < 1 || k > dsa::kMaxK) return DSA_ERR_BAD_K;
+  if (row_stride < 1) return DSA_ERR_BAD_STRIDE;
+  if (num_rows < 0) return DSA_ERR_BAD_ROWS;
+  dsa::DeviceInfo d;
+  const int rc = dsa::current_device(&d);
+  if (rc != DSA_OK) return rc;
+  int cs;
+  int64_t g;
+  dsa::plan(d, num_rows, row_stride, &cs, &g);
+  if (cluster_size) *cluster_size = cs;
+  if (grid) *grid = static_cast<int32_t>(g > 0x7fffffff ? 0x7fffffff : g);
+  return DSA_OK;
+}
+
+DSA_EXPORT int dsa_topk_device_status(uint32_t* status, int clear) {
+  unsigned int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess || cudaMemcpyFromSymbol(&v, dsa::g_status, sizeof(v)) != cudaSuccess) {
+    cudaGetLastError();
+    return DSA_ERR_LAUNCH;
+  }
+  if (status) *status = v;
+  if (clear) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(dsa::g_status, &z, sizeof(z)) != cudaSuccess) {
+      cudaGetLastError();
+      return DSA_ERR_LAUNCH;
+    }
+  }
+  return DSA_OK;
+}
+
+DSA_EXPORT const char* dsa_topk_strerror(int code) {
+  switch (code) {
+    case DSA_OK: return "success";
+    case DSA_ERR_NULL_POINTER: return "a required pointer is NULL";
+    case DSA_ERR_BAD_K: return "k must be in [1, 2048]";
+    case DSA_ERR_BAD_STRIDE: return "row_stride must be >= 1";
+    case DSA_ERR_BAD_ROWS: return "num_rows must be >= 0";
+    case DSA_ERR_OVERFLOW: return "sizes overflow int64 / the launch grid";
+    case DSA_ERR_MISALIGNED: return "a pointer is not 4-byte aligned";
+    case DSA_ERR_NO_DEVICE: return "no current CUDA device of compute capability 10.x (sm_100)";
+    case DSA_ERR_LAUNCH: return "the CUDA runtime rejected a launch or copy";
+    case DSA_ERR_CONFIG: return "kernel attribute set-up failed on this device";
+    default: return "unknown dsa_topk error code";
+  }
+}
+
+DSA_EXPORT int dsa_topk_version(void) { return 100; }

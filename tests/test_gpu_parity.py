@@ -1,0 +1,287 @@
+"""GPU parity: the CUDA path against the CPU oracle, index for index.
+
+All inputs are seeded. Every comparison is exact (integer outputs). Calls go
+through the C ABI (ctypes) with torch used only for device memory and streams.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from tests.topk_checks import check_all
+
+pytestmark = pytest.mark.gpu
+
+CANARY = -123456789
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import sparse_attention_indexer_strided_b200 as m
+    m.device_status(clear=True)
+    return m
+
+
+def run_gpu(dsa, logits2d, lengths, k, base_offset=0, stride=None):
+    """Lay rows out on the device at `stride` (default: the array's own),
+    starting `base_offset` floats into the buffer, call dsa_topk through the
+    C ABI and return the [rows, k] result. Guard words around the output must
+    survive."""
+    logits2d = np.asarray(logits2d, np.float32)
+    rows, width = logits2d.shape
+    stride = width if stride is None else stride
+    assert stride >= width or rows <= 1
+    buf = torch.full((base_offset + max(rows, 1) * stride + 8,), float("inf"), dtype=torch.float32)
+    view = buf[base_offset: base_offset + rows * stride].view(rows, stride) if rows else None
+    if rows:
+        view[:, :width] = torch.from_numpy(logits2d)
+    d_buf = buf.cuda()
+    d_len = torch.from_numpy(np.asarray(lengths, np.int32).copy()).cuda()
+    d_out = torch.full((rows * k + 64,), CANARY, dtype=torch.int32, device="cuda")
+    out_ptr = d_out.data_ptr() + 32 * 4
+    rc = dsa.lib.dsa_topk(d_buf.data_ptr() + 4 * base_offset, stride, d_len.data_ptr(), rows, k, out_ptr,
+                          torch.cuda.current_stream().cuda_stream)
+    assert rc == 0, dsa.strerror(rc)
+    torch.cuda.synchronize()
+    o = d_out.cpu().numpy()
+    assert np.all(o[:32] == CANARY) and np.all(o[32 + rows * k:] == CANARY), "output guard words overwritten"
+    return o[32:32 + rows * k].reshape(rows, k)
+
+
+def assert_parity(oracle_mod, dsa, logits2d, lengths, k, **kw):
+    got = run_gpu(dsa, logits2d, lengths, k, **kw)
+    exp = oracle_mod.topk(logits2d, lengths, k)
+    if not np.array_equal(got, exp):
+        bad = np.nonzero(np.any(got != exp, axis=1))[0]
+        r = bad[0]
+        j = np.nonzero(got[r] != exp[r])[0][0]
+        raise AssertionError("mismatch in %d rows; first row %d (L=%d) at t=%d: gpu %s oracle %s" % (
+            len(bad), r, lengths[r], j, got[r, j:j + 6], exp[r, j:j + 6]))
+    return got
+
+
+# ------------------------------------------------------------ the 5 workloads
+@pytest.mark.parametrize("name", ["tiny", "decode", "cluster", "ties"])
+def test_workload_full_parity(oracle_mod, dsa, name):
+    wl = workloads.make(name)
+    got = assert_parity(oracle_mod, dsa, wl.logits, wl.lengths, wl.k)
+    check_all(wl.logits, wl.lengths, wl.k, got)
+
+
+def test_prefill_full_size_sampled_rows(oracle_mod, dsa):
+    """Full prefill batch on the GPU; the oracle checks a spread of rows."""
+    wl = workloads.make("prefill")
+    got = run_gpu(dsa, wl.logits, wl.lengths, wl.k)
+    rng = np.random.default_rng(99)
+    rows = sorted(set([0, 1, 2, 147, 148, 2047, 4094, 4095] + rng.choice(4096, 40, replace=False).tolist()))
+    exp = oracle_mod.topk(wl.logits[rows], wl.lengths[rows], wl.k)
+    np.testing.assert_array_equal(got[rows], exp)
+    # every row: in-range, distinct, no padding needed (L > k)
+    assert got.min() >= 0 and np.all(got < wl.lengths[:, None])
+    srt = np.sort(got, axis=1)
+    assert np.all(srt[:, 1:] != srt[:, :-1])
+
+
+def test_plan_choices(dsa):
+    """Dispatch picks the cluster path for few long rows only."""
+    assert dsa.plan(4096, 131072, 2048)[0] == 1
+    assert dsa.plan(256, 131328, 2048)[0] == 1
+    assert dsa.plan(4, 4096, 512)[0] == 1
+    assert dsa.plan(4, 900096, 1024)[0] > 1
+    assert dsa.plan(64, 65536, 2048)[0] > 1
+
+
+# ------------------------------------------------------------------ k sweep
+LEN_MIX = [0, 1, 2, 30, 31, 32, 254, 255, 511, 512, 513, 1023, 1024, 1025, 2047, 2048, 2049,
+           4095, 4096, 4097, 8191, 8192, 8193, 10239, 10240, 10241, 12288, 20000, 33333]
+
+
+@pytest.mark.parametrize("k", [1, 31, 255, 512, 1023, 1024, 2047, 2048])
+def test_k_sweep_many_rows(oracle_mod, dsa, k):
+    rng = np.random.default_rng(1000 + k)
+    stride = max(LEN_MIX) + 3
+    rows = len(LEN_MIX) * 6  # >= SM count: one CTA per row
+    L = np.array((LEN_MIX * 6)[:rows], np.int32)
+    x = rng.standard_normal((rows, stride)).astype(np.float32)
+    x[1::3] = np.round(x[1::3] * 4) / 4  # coarse grid: ties at the threshold
+    assert_parity(oracle_mod, dsa, x, L, k)
+
+
+@pytest.mark.parametrize("k", [1, 255, 1024, 2048])
+def test_k_sweep_cluster_path(oracle_mod, dsa, k):
+    rng = np.random.default_rng(2000 + k)
+    stride = 300000
+    L = np.array([300000, 123457, 20000, 2047, 0, 299999], np.int32)
+    x = rng.standard_normal((len(L), stride)).astype(np.float32)
+    x[2] = np.round(x[2] * 2) / 2
+    assert dsa.plan(len(L), stride, k)[0] > 1
+    assert_parity(oracle_mod, dsa, x, L, k)
+
+
+# --------------------------------------------------------- layout and poison
+@pytest.mark.parametrize("extra,offset", [(0, 0), (1, 0), (2, 1), (3, 3), (5, 2), (256, 0)])
+def test_unaligned_strides_and_bases(oracle_mod, dsa, extra, offset):
+    rng = np.random.default_rng(extra * 10 + offset)
+    L = np.array([5000, 4096, 17, 9000, 4093, 1, 0, 8195] * 20, np.int32)
+    stride = int(L.max()) + extra
+    x = rng.standard_normal((len(L), stride)).astype(np.float32)
+    assert_parity(oracle_mod, dsa, x, L, 512, base_offset=offset)
+
+
+@pytest.mark.parametrize("offset", [0, 1, 2, 3])
+def test_unaligned_cluster_path(oracle_mod, dsa, offset):
+    rng = np.random.default_rng(77 + offset)
+    L = np.array([250001, 199999, 250003], np.int32)
+    stride = 250003 + offset
+    x = rng.standard_normal((3, stride)).astype(np.float32)
+    assert_parity(oracle_mod, dsa, x, L, 1024, base_offset=offset)
+
+
+@pytest.mark.parametrize("poison", [np.inf, np.nan, -np.inf, 3.0e38])
+def test_padding_is_never_read(oracle_mod, dsa, poison):
+    wl = workloads.make_rows("decode", [0, 1, 2, 3, 4, 5, 6, 7])
+    a = np.full_like(wl.logits, poison)
+    for i in range(wl.num_rows):
+        a[i, :wl.lengths[i]] = wl.logits[i, :wl.lengths[i]]
+    base = run_gpu(dsa, wl.logits, wl.lengths, wl.k)
+    got = run_gpu(dsa, a, wl.lengths, wl.k)
+    np.testing.assert_array_equal(got, base)
+    np.testing.assert_array_equal(got, oracle_mod.topk(wl.logits, wl.lengths, wl.k))
+
+
+def test_stride_invariance_on_gpu(dsa):
+    wl = workloads.make_rows("decode", range(16))
+    base = run_gpu(dsa, wl.logits, wl.lengths, wl.k)
+    Lmax = int(wl.lengths.max())
+    for stride in (Lmax, Lmax + 3, 2 * Lmax + 1):
+        a = np.ascontiguousarray(wl.logits[:, :Lmax])
+        np.testing.assert_array_equal(run_gpu(dsa, a, wl.lengths, wl.k, stride=stride), base)
+
+
+def test_lengths_are_clamped(oracle_mod, dsa):
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((6, 3000)).astype(np.float32)
+    L = np.array([-5, 0, 3000, 3001, 2 ** 31 - 1, 1500], np.int32)
+    assert_parity(oracle_mod, dsa, x, L, 256)
+
+
+# ------------------------------------------------------------ value patterns
+def _special_rows(rng, rows, width):
+    pool = np.array([np.nan, np.inf, -np.inf, 0.0, -0.0, 1.0, -1.0, 2.5], np.float32)
+    x = rng.standard_normal((rows, width)).astype(np.float32)
+    mask = rng.random((rows, width)) < 0.05
+    x[mask] = pool[rng.integers(0, len(pool), mask.sum())]
+    return x
+
+
+def test_special_values(oracle_mod, dsa):
+    rng = np.random.default_rng(8)
+    x = _special_rows(rng, 200, 9000)
+    x[3, :] = np.nan
+    x[4, :] = -np.inf
+    x[5, :] = -0.0
+    x[6, ::2] = 0.0
+    x[7, :] = np.inf
+    L = rng.integers(0, 9001, 200).astype(np.int32)
+    L[3:8] = 9000
+    assert_parity(oracle_mod, dsa, x, L, 2048)
+
+
+def test_special_values_cluster(oracle_mod, dsa):
+    rng = np.random.default_rng(9)
+    x = _special_rows(rng, 3, 200000)
+    x[1, 150000:] = np.nan
+    x[2, :] = -0.0
+    x[2, 199990] = 0.0
+    L = np.array([200000, 200000, 200000], np.int32)
+    assert_parity(oracle_mod, dsa, x, L, 1024)
+
+
+@pytest.mark.parametrize("pattern", ["increasing", "decreasing", "all_equal", "two_levels", "sawtooth"])
+@pytest.mark.parametrize("rows", [160, 3])
+def test_adversarial_orders(oracle_mod, dsa, pattern, rows):
+    width = 150000 if rows == 3 else 40000
+    j = np.arange(width, dtype=np.float64)
+    if pattern == "increasing":
+        row = j
+    elif pattern == "decreasing":
+        row = -j
+    elif pattern == "all_equal":
+        row = np.zeros(width)
+    elif pattern == "two_levels":
+        row = (j % 7 == 0).astype(np.float64)
+    else:
+        row = j % 5000
+    x = np.tile(row.astype(np.float32), (rows, 1))
+    L = np.full(rows, width, np.int32)
+    L[::2] = width - 7
+    assert_parity(oracle_mod, dsa, x, L, 2048)
+
+
+def test_heavy_ties_cluster_exact_path(oracle_mod, dsa):
+    """Few levels across a cluster-split row: the merge must split the tied
+    threshold level across ranks in index order."""
+    rng = np.random.default_rng(12)
+    x = (rng.integers(0, 3, (4, 400000)) * 1.0).astype(np.float32)
+    L = np.array([400000, 399999, 262145, 400000], np.int32)
+    assert_parity(oracle_mod, dsa, x, L, 2048)
+    assert_parity(oracle_mod, dsa, x, L, 7)
+
+
+# ------------------------------------------------------------ execution model
+def test_repeat_calls_are_deterministic(dsa):
+    wl = workloads.make("decode")
+    a = run_gpu(dsa, wl.logits, wl.lengths, wl.k)
+    for _ in range(3):
+        np.testing.assert_array_equal(run_gpu(dsa, wl.logits, wl.lengths, wl.k), a)
+
+
+def test_cuda_graph_replay(oracle_mod, dsa):
+    wl = workloads.make("decode")
+    logits = torch.from_numpy(wl.logits).cuda()
+    lengths = torch.from_numpy(wl.lengths).cuda()
+    out = torch.empty((wl.num_rows, wl.k), dtype=torch.int32, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        dsa.dsa_topk(logits, lengths, wl.k, out=out)  # uncaptured first call (attributes)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(3):
+            dsa.dsa_topk(logits, lengths, wl.k, out=out)
+    exp = oracle_mod.topk(wl.logits, wl.lengths, wl.k)
+    for _ in range(5):
+        out.fill_(-7)
+        g.replay()
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(out.cpu().numpy(), exp)
+    del g
+
+
+def test_torch_binding_uses_stride0(oracle_mod, dsa):
+    """A sliced (non-contiguous) view is read at its row stride."""
+    wl = workloads.make_rows("tiny", range(4))
+    full = torch.from_numpy(wl.logits).cuda()          # [4, 4096]
+    view = full[:, :4000]                               # stride(0) = 4096, size(1) = 4000
+    assert view.stride(0) == 4096 and not view.is_contiguous()
+    out = dsa.dsa_topk(view, torch.from_numpy(wl.lengths).cuda(), wl.k)
+    np.testing.assert_array_equal(out.cpu().numpy(), oracle_mod.topk(wl.logits, wl.lengths, wl.k))
+
+
+def test_host_buffer_entry_point(oracle_mod, dsa):
+    wl = workloads.make("tiny")
+    h_logits = torch.from_numpy(wl.logits).pin_memory()
+    h_len = torch.from_numpy(wl.lengths).pin_memory()
+    h_out = torch.empty((wl.num_rows, wl.k), dtype=torch.int32).pin_memory()
+    d_logits = torch.empty(wl.logits.size, dtype=torch.float32, device="cuda")
+    d_len = torch.empty(wl.num_rows, dtype=torch.int32, device="cuda")
+    d_out = torch.empty(wl.num_rows * wl.k, dtype=torch.int32, device="cuda")
+    dsa.dsa_topk_host(h_logits, h_len, wl.k, h_out, d_logits, d_len, d_out)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(h_out.numpy(), oracle_mod.topk(wl.logits, wl.lengths, wl.k))
+
+
+def test_no_device_side_timeouts(dsa):
+    assert dsa.device_status() == 0
