@@ -48,18 +48,23 @@
 
 namespace dsa {
 
-constexpr int kNumConsumerWarps = 16;
-constexpr int kConsumerThreads = kNumConsumerWarps * 32;       // 512
-constexpr int kThreads = kConsumerThreads + 32;                // + producer warp
-constexpr int kStageElems = 4096;                              // 16 KB per stage
+constexpr int kNumConsumerWarps = 8;                           // every warp consumes
+constexpr int kConsumerThreads = kNumConsumerWarps * 32;       // 256
+constexpr int kThreads = kConsumerThreads;
+constexpr int kBlocksPerSM = 2;                                // one CTA selects/sorts while the other streams
+constexpr int kStageElems = kNumConsumerWarps * 512;           // 16 KB per stage
 constexpr uint32_t kStageBytes = kStageElems * 4;
-constexpr int kStages = 8;                                     // 128 KB ring
+constexpr int kStages = 3;                                     // 48 KB ring
+constexpr int kWarpStageElems = kStageElems / kNumConsumerWarps;  // 512 = 4 groups x 32 lanes x float4
 constexpr int kMaxK = DSA_TOPK_MAX_K;
-constexpr int kCap = kMaxK + 2 * kStageElems;                  // candidate buffer entries
+constexpr int kCap = kMaxK + kStageElems;                      // candidate buffer entries
 constexpr int kGatherOff = kMaxK;                              // cluster gather region
 constexpr int kGatherCap = kCap - kGatherOff;
 constexpr int kSortCountOff = 2 * kMaxK;                       // sort counters alias free space
 constexpr int kMaxEntriesPerThread = (kCap + kConsumerThreads - 1) / kConsumerThreads;
+constexpr int kStage2 = 192;  // per-warp staging entries for one stage's survivors
+constexpr int kSortItemsPerWarp = kMaxK / kNumConsumerWarps;   // 256
+constexpr int kSortSlots = kSortItemsPerWarp / 32;              // 8 per lane
 constexpr uint32_t kNanKey = 0xFFC00000u;  // key of the canonical quiet NaN
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr unsigned long long kWaitLimitNs = 500000000ull;     // 0.5 s per pipeline wait
@@ -72,8 +77,22 @@ constexpr unsigned kStatusSelectBroken = 2u;  // a radix round lost its invarian
 static_assert(kSortCountOff + kNumConsumerWarps * 256 <= kCap, "sort counters must fit");
 static_assert(kGatherCap >= kMaxK, "gather region must hold k entries");
 static_assert(kCap - kMaxK >= kStageElems, "a stage must fit after a compaction");
+static_assert(kWarpStageElems == 4 * 32 * 4, "a warp covers 4 float4 groups per stage");
+static_assert(kConsumerThreads >= 256, "digit-parallel steps use one thread per 8-bit digit");
 
-enum Mode : int { kAcceptAll = 0, kFilter = 1, kRejectAll = 2 };
+// Stream filter: kAcceptAll keeps every valid entry; kAbove keeps key > T (T is
+// the exact k-th key of what was seen); kAtLeast keeps key >= T (T is a lower
+// estimate taken from the previous row); kRejectAll keeps nothing (T is NaN).
+enum Mode : int { kAcceptAll = 0, kAbove = 1, kAtLeast = 2, kRejectAll = 3 };
+
+// A work item is the slice [c0, c1) of one row. Its bytes are fetched as the
+// 16-byte aligned span that covers them; entries outside [c0, c1) are masked.
+struct Span {
+  const char* src;   // 16-byte aligned start
+  int64_t j0;        // row-local index of the first float of the span
+  uint64_t bytes;    // span length, multiple of 16
+  int nst;           // stages
+};
 
 struct __align__(128) Smem {
   float ring[kStages][kStageElems];
@@ -87,10 +106,12 @@ struct __align__(128) Smem {
   uint32_t pub[8];  // published to the cluster
   uint32_t bc[8];
   uint32_t skip[4];
+  uint32_t small[32];
+  uint32_t stg_key[kNumConsumerWarps][kStage2];
+  uint32_t stg_idx[kNumConsumerWarps][kStage2];
   unsigned long long full[kStages];
-  unsigned long long empty[kStages];
 };
-static_assert(sizeof(Smem) <= 232448, "shared memory budget (227 KB)");
+static_assert(sizeof(Smem) <= 232448 / kBlocksPerSM - 1024, "shared memory budget per CTA");
 
 __device__ unsigned int g_status;  // sticky status bits, see kStatus*
 
@@ -103,6 +124,11 @@ __device__ __forceinline__ void mbar_init(unsigned long long* bar, uint32_t coun
 }
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// Orders this thread's earlier generic-proxy shared-memory accesses (made
+// visible by a preceding barrier) before a following TMA write.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
@@ -147,9 +173,7 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
-__device__ __forceinline__ void bar_consumers() {
-  asm volatile("bar.sync 1, %0;" ::"r"(kConsumerThreads) : "memory");
-}
+__device__ __forceinline__ void bar_consumers() { __syncthreads(); }
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
@@ -206,15 +230,6 @@ __device__ __forceinline__ float from_key(uint32_t key) {
 }
 
 // ------------------------------------------------------------ row geometry
-// A work item is the slice [c0, c1) of one row. Its bytes are fetched as the
-// 16-byte aligned span that covers them; entries outside [c0, c1) are masked.
-struct Span {
-  const char* src;   // 16-byte aligned start
-  int64_t j0;        // row-local index of the first float of the span
-  uint64_t bytes;    // span length, multiple of 16
-  int nst;           // stages
-};
-
 __device__ __forceinline__ Span make_span(const float* row, int64_t c0, int64_t c1) {
   Span sp;
   if (c1 <= c0) {
@@ -244,20 +259,57 @@ __device__ __forceinline__ int64_t clamp_len(const int32_t* lengths, int64_t row
   return L;
 }
 
-// Producer: issue every stage of one work item into the ring.
-__device__ __forceinline__ void produce_item(Smem& s, const Span& sp, int& stage, uint32_t& phase) {
-  for (int t = 0; t < sp.nst; ++t) {
-    mbar_wait(&s.empty[stage], phase ^ 1u);
-    const uint64_t off = static_cast<uint64_t>(t) * kStageBytes;
-    const uint64_t rem = sp.bytes - off;
-    const uint32_t bytes = rem < kStageBytes ? static_cast<uint32_t>(rem) : kStageBytes;
-    mbar_arrive_expect_tx(&s.full[stage], bytes);
-    bulk_g2s(&s.ring[stage][0], sp.src + off, bytes, &s.full[stage]);
-    if (++stage == kStages) {
-      stage = 0;
-      phase ^= 1u;
-    }
+// Producer cursor, advanced by thread 0 only. It walks the same sequence of
+// (work item, stage) pairs as the consumers, kStages stages ahead of them: a
+// stage is issued into the ring slot that the consumers released at the
+// barrier that ended the stage kStages before it.
+
+struct Producer {
+  int64_t row;          // current work item
+  const char* src;      // its 16-byte aligned span start
+  uint32_t nst, t;      // its stage count, next stage to issue
+  uint32_t last_bytes;  // bytes of its last stage
+  uint32_t g;           // stages issued so far (slot = g % kStages)
+};
+
+struct ItemSource {
+  const float* logits;
+  const int32_t* lengths;
+  int64_t row_stride, row_end, row_step;
+  int64_t c0, c1;  // slice of the row; c1 < 0: the whole valid row
+};
+
+__device__ __forceinline__ void producer_set_item(Producer& p, const ItemSource& is) {
+  p.t = 0;
+  p.nst = 0;
+  if (p.row >= is.row_end) return;
+  const int64_t L = clamp_len(is.lengths, p.row, is.row_stride);
+  const int64_t c1 = is.c1 < 0 ? L : min64(is.c1, L);
+  const Span sp = make_span(is.logits + p.row * is.row_stride, min64(is.c0, c1), c1);
+  p.src = sp.src;
+  p.nst = static_cast<uint32_t>(sp.nst);
+  p.last_bytes = sp.nst ? static_cast<uint32_t>(sp.bytes - static_cast<uint64_t>(sp.nst - 1) * kStageBytes) : 0u;
+}
+
+__device__ __forceinline__ uint32_t stage_bytes(const Producer& p, uint32_t t) {
+  return t + 1 == p.nst ? p.last_bytes : kStageBytes;
+}
+
+// Issue the next stage, if any remains.
+__device__ __forceinline__ void producer_issue(Smem& s, Producer& p, const ItemSource& is) {
+  while (p.t >= p.nst) {
+    if (p.row >= is.row_end) return;
+    p.row += is.row_step;
+    producer_set_item(p, is);
   }
+  const int slot = static_cast<int>(p.g % kStages);
+  const uint32_t bytes = stage_bytes(p, p.t);
+  const char* src = p.src + static_cast<uint64_t>(p.t) * kStageBytes;
+  fence_proxy_async();
+  mbar_arrive_expect_tx(&s.full[slot], bytes);
+  bulk_g2s(&s.ring[slot][0], src, bytes, &s.full[slot]);
+  ++p.t;
+  ++p.g;
 }
 
 // ------------------------------------------------------ block-level helpers
@@ -337,21 +389,33 @@ __device__ __forceinline__ int window_shift(uint32_t lo, uint32_t hi) {
 }
 
 // Histogram of keys in [lo, hi] over entries [base, base+n) into hist[256]
-// (already zeroed). Lanes with the same digit combine into one atomic.
+// (already zeroed). Each thread walks its strided entries and adds a run of
+// equal digits with one atomic, so heavily tied keys cost few atomics.
 __device__ __forceinline__ void histogram(const Smem& s, uint32_t* hist, int base, int n, uint32_t lo, uint32_t hi,
                                           int sh, int tid) {
-  const int lane = tid & 31;
-  const int iters = (n + kConsumerThreads - 1) / kConsumerThreads;
-  for (int it = 0; it < iters; ++it) {
-    const int e = it * kConsumerThreads + tid;
-    uint32_t d = 0xFFFFFFFFu;
-    if (e < n) {
-      const uint32_t key = s.ckey[base + e];
-      if (key >= lo && key <= hi) d = (key >> sh) & 255u;
+  uint32_t cur = 0xFFFFFFFFu, run = 0;
+  for (int e = tid; e < n; e += kConsumerThreads) {
+    const uint32_t key = s.ckey[base + e];
+    if (key < lo || key > hi) continue;
+    const uint32_t d = (key >> sh) & 255u;
+    if (d != cur) {
+      if (run) atomicAdd(&hist[cur], run);
+      cur = d;
+      run = 0;
     }
-    const uint32_t peers = __match_any_sync(kFull, d);
-    if (d != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[d], static_cast<uint32_t>(__popc(peers)));
+    ++run;
   }
+  if (run) atomicAdd(&hist[cur], run);
+}
+
+// Exact need-th largest key among the <= 32 keys in [lo, hi] (warp 0). Every
+// lane holds one key (or 0, below any real key); returns the largest key x with
+// #{keys >= x} >= need.
+__device__ __forceinline__ uint32_t small_kth(uint32_t mine, uint32_t need) {
+  uint32_t ge = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) ge += __shfl_sync(kFull, mine, j) >= mine;
+  return __reduce_max_sync(kFull, (mine != 0u && ge >= need) ? mine : 0u);
 }
 
 // Stable selection of entries [base, base+n): keep key > T, plus the first
@@ -413,11 +477,11 @@ __device__ void stable_keep(Smem& s, int base, int n, uint32_t T, uint32_t need_
 }
 
 // Counts of keys > T and == T over entries [0, n) (block-wide, consumers).
-__device__ void count_gt_eq(Smem& s, int n, uint32_t T, uint32_t& ngt, uint32_t& neq, int tid) {
+__device__ void count_gt_eq(Smem& s, int base, int n, uint32_t T, uint32_t& ngt, uint32_t& neq, int tid) {
   const int w = tid >> 5, lane = tid & 31;
   uint32_t g = 0, q = 0;
   for (int e = tid; e < n; e += kConsumerThreads) {
-    const uint32_t key = s.ckey[e];
+    const uint32_t key = s.ckey[base + e];
     g += key > T;
     q += key == T;
   }
@@ -435,7 +499,10 @@ __device__ void count_gt_eq(Smem& s, int n, uint32_t T, uint32_t& ngt, uint32_t&
 
 // Exact selection: entries [base, base+n), n > k. Keeps the k largest keys in
 // place, in index order, ties to the lowest index. Returns the k-th largest key.
-__device__ uint32_t select_topk(Smem& s, int base, int n, int k, int tid) {
+// Radix rounds narrow [lo, hi] (8-bit windows below the highest bit where lo
+// and hi differ); once the bucket holding the k-th key has <= 32 entries, warp 0
+// finishes it directly.
+__device__ __noinline__ uint32_t select_topk(Smem& s, int base, int n, int k, int tid) {
   const int w = tid >> 5, lane = tid & 31;
   const MinMax r = block_minmax(s, base, n, tid);
   uint32_t lo = r.mn, hi = r.mx, need = static_cast<uint32_t>(k);
@@ -446,21 +513,44 @@ __device__ uint32_t select_topk(Smem& s, int base, int n, int k, int tid) {
     }
     const int sh = window_shift(lo, hi);
     if (tid < 256) s.hist[tid] = 0u;
-    if (tid == 0) s.bc[0] = 0xFFFFFFFFu;
-    bar_consumers();
+    if (tid == 0) {
+      s.bc[0] = 0xFFFFFFFFu;
+      s.bc[2] = 0u;
+    }
+    __syncthreads();
     histogram(s, s.hist, base, n, lo, hi, sh, tid);
-    bar_consumers();
+    __syncthreads();
     if (w == 0) find_bucket_warp0(s.hist, need, s.bc, lane);
-    bar_consumers();
-    if (s.bc[0] == 0xFFFFFFFFu) {  // no bucket holds the need-th key
+    __syncthreads();
+    const uint32_t b = s.bc[0], above_b = s.bc[1];
+    if (b == 0xFFFFFFFFu) {  // no bucket holds the need-th key
       if (tid == 0) atomicOr(&g_status, kStatusSelectBroken);
-      bar_consumers();
       break;
     }
-    const uint32_t b = s.bc[0], above_b = s.bc[1];
+    const uint32_t in_bucket = s.hist[b];
     need -= above_b;
     narrow(lo, hi, sh, b);
-    bar_consumers();  // bc / hist reused by the next round
+    if (in_bucket <= 32u && lo != hi) {
+      // gather the bucket's keys (order irrelevant) and finish in one warp
+      for (int e = tid; e < n; e += kConsumerThreads) {
+        const uint32_t key = s.ckey[base + e];
+        if (key >= lo && key <= hi) s.small[atomicAdd(&s.bc[2], 1u)] = key;
+      }
+      __syncthreads();
+      if (w == 0) {
+        const uint32_t mine = lane < static_cast<int>(in_bucket) ? s.small[lane] : 0u;
+        const uint32_t t = small_kth(mine, need);
+        const uint32_t above = __popc(__ballot_sync(kFull, mine > t));
+        if (lane == 0) {
+          s.bc[3] = t;
+          s.bc[4] = need - above;
+        }
+      }
+      __syncthreads();
+      lo = hi = s.bc[3];
+      need = s.bc[4];
+    }
+    __syncthreads();  // bc / hist / small reused by the next round
   }
   stable_keep<false>(s, base, n, lo, need, 0u, 0u, 0u, tid);
   return lo;
@@ -468,65 +558,80 @@ __device__ uint32_t select_topk(Smem& s, int base, int n, int k, int tid) {
 
 // Stable LSD radix sort of entries [src, src+m) (m <= kMaxK) by key
 // descending, using [alt, alt+m) as the other buffer. Ties keep buffer order.
-// Returns the base that holds the sorted entries.
-__device__ int sort_desc(Smem& s, int src, int alt, int m, int tid) {
+// Returns the base that holds the sorted entries. Bytes of the key above the
+// highest bit where the smallest and largest keys differ are equal for every
+// entry, so only the passes below it run. Within a warp, lanes holding the
+// same digit are found with eight ballots (one per digit bit).
+__device__ __noinline__ int sort_desc(Smem& s, int src, int alt, int m, int tid) {
   const int w = tid >> 5, lane = tid & 31;
+  if (m <= 1) return src;
+  const MinMax mm = block_minmax(s, src, m, tid);
+  if (mm.mn == mm.mx) return src;
+  const int passes = (31 - __clz(mm.mn ^ mm.mx)) / 8 + 1;
   uint32_t* wcnt = s.ckey + kSortCountOff;  // [warp][256]
-  if (tid < 4) s.skip[tid] = 0u;
   const uint32_t lt = lanemask_lt();
-  for (int pass = 0; pass < 4; ++pass) {
+  for (int pass = 0; pass < passes; ++pass) {
     const int sh = pass * 8;
-    for (int i = tid; i < kNumConsumerWarps * 256; i += kConsumerThreads) wcnt[i] = 0u;
-    bar_consumers();
-    uint32_t dig[4], lp[4];
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int item = w * 128 + it * 32 + lane;
+    for (int i = 0; i < 8; ++i) wcnt[w * 256 + i * 32 + lane] = 0u;
+    __syncwarp();
+    uint32_t dig[kSortSlots], lp[kSortSlots];
+#pragma unroll
+    for (int it = 0; it < kSortSlots; ++it) {
+      const int item = w * kSortItemsPerWarp + it * 32 + lane;
       const bool v = item < m;
-      const uint32_t d = v ? ((~s.ckey[src + item]) >> sh) & 255u : 0xFFFFFFFFu;
-      const uint32_t peers = __match_any_sync(kFull, d);
+      const uint32_t d = v ? ((~s.ckey[src + item]) >> sh) & 255u : 0u;
+      uint32_t peers = __ballot_sync(kFull, v);
+#pragma unroll
+      for (int bit = 0; bit < 8; ++bit) {
+        const uint32_t bb = __ballot_sync(kFull, (d >> bit) & 1u);
+        peers &= ((d >> bit) & 1u) ? bb : ~bb;
+      }
       const uint32_t c = v ? wcnt[w * 256 + d] : 0u;
       __syncwarp();
-      if (v && lane == __ffs(peers) - 1) wcnt[w * 256 + d] = c + __popc(peers);
+      if (v && (peers & lt) == 0u) wcnt[w * 256 + d] = c + __popc(peers);
       __syncwarp();
       dig[it] = d;
       lp[it] = c + __popc(peers & lt);
     }
-    bar_consumers();
-    uint32_t tot = 0, incl = 0;
+    __syncthreads();
+    // digit-major, warp-minor exclusive prefix: thread t < 256 owns digit t
+    uint32_t tot = 0, incl = 0, c[kNumConsumerWarps];
     if (tid < 256) {
+#pragma unroll
+      for (int ww = 0; ww < kNumConsumerWarps; ++ww) c[ww] = wcnt[ww * 256 + tid];
+#pragma unroll
       for (int ww = 0; ww < kNumConsumerWarps; ++ww) {
-        const uint32_t c = wcnt[ww * 256 + tid];
-        wcnt[ww * 256 + tid] = tot;
-        tot += c;
+        const uint32_t x = c[ww];
+        c[ww] = tot;
+        tot += x;
       }
-      if (tot == static_cast<uint32_t>(m)) s.skip[pass] = 1u;
       incl = tot;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += v;
+        const uint32_t y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
       }
       if (lane == 31) s.red[4][w] = incl;
     }
-    bar_consumers();
+    __syncthreads();
     if (tid < 256) {
       uint32_t dbase = incl - tot;
       for (int ww = 0; ww < w; ++ww) dbase += s.red[4][ww];
-      for (int ww = 0; ww < kNumConsumerWarps; ++ww) wcnt[ww * 256 + tid] += dbase;
-    }
-    bar_consumers();
-    if (s.skip[pass]) continue;  // every entry has the same digit: order unchanged
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int item = w * 128 + it * 32 + lane;
+      for (int ww = 0; ww < kNumConsumerWarps; ++ww) wcnt[ww * 256 + tid] = c[ww] + dbase;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < kSortSlots; ++it) {
+      const int item = w * kSortItemsPerWarp + it * 32 + lane;
       if (item < m) {
         const uint32_t dst = wcnt[w * 256 + dig[it]] + lp[it];
         s.ckey[alt + dst] = s.ckey[src + item];
         s.cidx[alt + dst] = s.cidx[src + item];
       }
     }
-    bar_consumers();
+    __syncthreads();
     const int t = src;
     src = alt;
     alt = t;
@@ -541,134 +646,278 @@ __device__ __forceinline__ void write_row(const Smem& s, int R, int m, int k, in
 
 // ------------------------------------------------------------ stream phase
 struct StreamState {
-  uint32_t count;  // candidates held (uniform across consumers)
+  uint32_t count;  // candidates held (uniform across threads)
   int mode;
-  float thr;       // from_key(T) when mode == kFilter
+  float thr;       // threshold value for kAbove / kAtLeast
   int par;         // wtot double-buffer parity
 };
 
-__device__ __forceinline__ void set_threshold(StreamState& st, uint32_t T) {
+__device__ __forceinline__ void set_exact_threshold(StreamState& st, uint32_t T) {
   if (T == kNanKey) {
     st.mode = kRejectAll;
   } else {
-    st.mode = kFilter;
+    st.mode = kAbove;
     st.thr = from_key(T);
   }
 }
 
-// Consume one stage: filter, append survivors in index order.
-__device__ __forceinline__ void consume_stage(Smem& s, StreamState& st, int stage, int64_t jbase, int64_t c0,
-                                              int64_t c1, int k, int tid) {
-  const int w = tid >> 5, lane = tid & 31;
-  const float* src = &s.ring[stage][0];
-  const int o0 = w * 256 + lane * 4, o1 = o0 + 128;
-  const float4 v0 = *reinterpret_cast<const float4*>(src + o0);
-  const float4 v1 = *reinterpret_cast<const float4*>(src + o1);
-  __syncwarp();
-  if (lane == 0) mbar_arrive(&s.empty[stage]);  // data is in registers: release the slot
+// The 16 values a thread looks at in one stage: group j is the float4 at
+// stage offset warp*512 + j*128 + lane*4 (coalesced, conflict-free reads).
+struct Lane16 {
+  float x[4][4];
+};
 
-  int64_t lo64 = c0 - jbase, hi64 = c1 - jbase;
+__device__ __forceinline__ int lane_offset(int w, int lane, int j) { return w * kWarpStageElems + j * 128 + lane * 4; }
+
+// v.x[b >> 2][b & 3] for a runtime b in [0, 16), as a select tree (keeps the
+// values in registers).
+__device__ __forceinline__ float pick16(const Lane16& v, int b) {
+  float q[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float lo = (b & 1) ? v.x[j][1] : v.x[j][0];
+    const float hi = (b & 1) ? v.x[j][3] : v.x[j][2];
+    q[j] = (b & 2) ? hi : lo;
+  }
+  const float lo = (b & 4) ? q[1] : q[0];
+  const float hi = (b & 4) ? q[3] : q[2];
+  return (b & 8) ? hi : lo;
+}
+
+// Filter one stage's values (in registers; `src` points at the same stage in
+// shared or global memory), then append the survivors to the candidate buffer
+// in index order. Index order inside a warp is (group, lane, component); one
+// warp scan over byte-packed per-group counts gives every survivor its rank r
+// in the warp. Before the stage barrier, lane r gathers the r-th survivor into
+// the warp's staging area (so lanes work on one survivor each instead of
+// looping over their own); after the barrier the staged entries are copied to
+// the candidate buffer behind the warps before it. `prod` (thread 0 only, may
+// be null) issues the next ring stage right after that barrier, which ends
+// every read of this stage's slot.
+__device__ __forceinline__ void consume_values(Smem& s, StreamState& st, const Lane16& v, const float* src,
+                                               int64_t jbase, int64_t c0, int64_t c1, int k, int tid, Producer* prod,
+                                               const ItemSource* is) {
+  const int w = tid >> 5, lane = tid & 31;
+  const int64_t lo64 = c0 - jbase, hi64 = c1 - jbase;
   const int lo = static_cast<int>(lo64 < 0 ? 0 : (lo64 > kStageElems ? kStageElems : lo64));
   const int hi = static_cast<int>(hi64 < 0 ? 0 : (hi64 > kStageElems ? kStageElems : hi64));
-  const float x0[4] = {v0.x, v0.y, v0.z, v0.w};
-  const float x1[4] = {v1.x, v1.y, v1.z, v1.w};
-  uint32_t f0 = 0, f1 = 0;
-  if (st.mode != kRejectAll) {
-    const bool all = st.mode == kAcceptAll;
-    const float thr = st.thr;
+  const bool filtering = st.mode == kAbove || st.mode == kAtLeast;
+  uint32_t F = 0;  // bit 4j+c: value x[j][c] survives
+  if (st.mode == kAbove) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const bool in0 = (o0 + c >= lo) && (o0 + c < hi);
-      const bool in1 = (o1 + c >= lo) && (o1 + c < hi);
-      const bool p0 = all || !(x0[c] <= thr);  // NaN passes any finite threshold
-      const bool p1 = all || !(x1[c] <= thr);
-      f0 |= static_cast<uint32_t>(in0 && p0) << c;
-      f1 |= static_cast<uint32_t>(in1 && p1) << c;
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) F |= static_cast<uint32_t>(!(v.x[j][c] <= st.thr)) << (4 * j + c);
+  } else if (st.mode == kAtLeast) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) F |= static_cast<uint32_t>(!(v.x[j][c] < st.thr)) << (4 * j + c);
+  }
+  if (filtering && (lo > 0 || hi < kStageElems)) {
+    // entries outside [c0, c1) (span head/tail, short last stage) never survive
+    uint32_t valid = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int o = lane_offset(w, lane, j) + c;
+        valid |= static_cast<uint32_t>(o >= lo && o < hi) << (4 * j + c);
+      }
+    F &= valid;
+  }
+  uint32_t excl = 0, tj[4] = {0, 0, 0, 0}, wt = 0;
+  if (filtering && __any_sync(kFull, F != 0u)) {
+    // per-group popcounts, one byte each (SWAR, no XU-pipe popc)
+    const uint32_t c2 = F - ((F >> 1) & 0x5555u);
+    const uint32_t c4 = (c2 & 0x3333u) + ((c2 >> 2) & 0x3333u);
+    const uint32_t packed = (c4 & 0xFu) | ((c4 & 0xF0u) << 4) | ((c4 & 0xF00u) << 8) | ((c4 & 0xF000u) << 12);
+    uint32_t incl = packed;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += t;  // each byte stays <= 128
+    }
+    excl = incl - packed;
+    const uint32_t tot = __shfl_sync(kFull, incl, 31);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tj[j] = (tot >> (8 * j)) & 0xFFu;
+    wt = tj[0] + tj[1] + tj[2] + tj[3];
+    if (wt <= static_cast<uint32_t>(kStage2)) {
+      // gather: lane r fetches the warp's r-th survivor (group-major order)
+      const uint32_t t0 = tj[0], t1 = t0 + tj[1], t2 = t1 + tj[2];
+      for (uint32_t r0 = 0; r0 < wt; r0 += 32) {
+        const uint32_t r = r0 + lane;
+        const int j = (r >= t0) + (r >= t1) + (r >= t2);
+        const uint32_t rj = r - (j == 0 ? 0u : (j == 1 ? t0 : (j == 2 ? t1 : t2)));
+        const int sj = 8 * j;
+        int l = 0;  // largest lane whose group-j exclusive prefix is <= rj
+#pragma unroll
+        for (int step = 16; step; step >>= 1) {
+          const uint32_t e = __shfl_sync(kFull, excl, l + step);
+          if (((e >> sj) & 0xFFu) <= rj) l += step;
+        }
+        const uint32_t el = (__shfl_sync(kFull, excl, l) >> sj) & 0xFFu;
+        uint32_t f = (__shfl_sync(kFull, F, l) >> (4 * j)) & 0xFu;
+        const uint32_t q = rj - el;  // q-th set bit of lane l's group-j nibble
+        if (q > 0) f &= f - 1u;
+        if (q > 1) f &= f - 1u;
+        if (q > 2) f &= f - 1u;
+        const int off = lane_offset(w, l, j) + (__ffs(f) - 1);
+        if (r < wt) {
+          s.stg_key[w][r] = to_key(src[off]);
+          s.stg_idx[w][r] = static_cast<uint32_t>(jbase + off);
+        }
+      }
     }
   }
-  uint32_t b0[4], b1[4];
-  uint32_t t0 = 0, t1 = 0;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    b0[c] = __ballot_sync(kFull, (f0 >> c) & 1u);
-    b1[c] = __ballot_sync(kFull, (f1 >> c) & 1u);
-    t0 += __popc(b0[c]);
-    t1 += __popc(b1[c]);
+  if (lane == 0) s.wtot[st.par][w] = wt;
+  __syncthreads();
+  if (prod) producer_issue(s, *prod, *is);
+  uint32_t pre = 0, tot = 0;
+  if (filtering) {
+    const uint32_t wv = lane < kNumConsumerWarps ? s.wtot[st.par][lane] : 0u;
+    pre = __reduce_add_sync(kFull, lane < w ? wv : 0u);
+    tot = __reduce_add_sync(kFull, wv);
+  } else if (st.mode == kAcceptAll) {
+    tot = static_cast<uint32_t>(hi > lo ? hi - lo : 0);
   }
-  if (lane == 0) s.wtot[st.par][w] = t0 + t1;
-  bar_consumers();
-  const uint32_t v = lane < kNumConsumerWarps ? s.wtot[st.par][lane] : 0u;
-  const uint32_t pre = __reduce_add_sync(kFull, lane < w ? v : 0u);
-  const uint32_t tot = __reduce_add_sync(kFull, v);
   st.par ^= 1;
   if (tot == 0) return;
   if (st.count + tot > static_cast<uint32_t>(kCap)) {
-    // Make room. Survivors of this stage passed the old threshold; appending
+    // Make room. This stage's survivors passed the old threshold; appending
     // them after the compaction keeps the buffer a superset of the winners.
     const uint32_t T = select_topk(s, 0, static_cast<int>(st.count), k, tid);
     st.count = static_cast<uint32_t>(k);
-    set_threshold(st, T);
+    set_exact_threshold(st, T);
   }
-  if (t0 + t1) {
-    const uint32_t lt = lanemask_lt();
-    uint32_t p0 = st.count + pre, p1 = st.count + pre + t0;
+  if (!filtering) {
+    // every entry in [lo, hi) survives: its rank is its offset
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      p0 += __popc(b0[c] & lt);
-      p1 += __popc(b1[c] & lt);
-    }
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if ((f0 >> c) & 1u) {
-        s.ckey[p0] = to_key(x0[c]);
-        s.cidx[p0] = static_cast<uint32_t>(jbase + o0 + c);
-        ++p0;
+      for (int c = 0; c < 4; ++c) {
+        const int o = lane_offset(w, lane, j) + c;
+        if (o >= lo && o < hi) {
+          const uint32_t p = st.count + static_cast<uint32_t>(o - lo);
+          s.ckey[p] = to_key(v.x[j][c]);
+          s.cidx[p] = static_cast<uint32_t>(jbase + o);
+        }
       }
+  } else if (wt <= static_cast<uint32_t>(kStage2)) {
+    const uint32_t base = st.count + pre;
+    for (uint32_t r = lane; r < wt; r += 32) {
+      s.ckey[base + r] = s.stg_key[w][r];
+      s.cidx[base + r] = s.stg_idx[w][r];
     }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if ((f1 >> c) & 1u) {
-        s.ckey[p1] = to_key(x1[c]);
-        s.cidx[p1] = static_cast<uint32_t>(jbase + o1 + c);
-        ++p1;
+  } else if (F) {
+    // more survivors than the staging area holds: each lane writes its own
+    const uint32_t base = st.count + pre;
+    const uint32_t g0 = base + (excl & 0xFFu);
+    const uint32_t g1 = base + tj[0] + ((excl >> 8) & 0xFFu);
+    const uint32_t g2 = base + tj[0] + tj[1] + ((excl >> 16) & 0xFFu);
+    const uint32_t g3 = base + tj[0] + tj[1] + tj[2] + (excl >> 24);
+    const int64_t jl = jbase + w * kWarpStageElems + lane * 4;
+    uint32_t rest = F, run = 0, gcur = 0;
+    int jcur = -1;
+    while (rest) {
+      const int b = __ffs(rest) - 1;
+      rest &= rest - 1u;
+      const int j = b >> 2;
+      if (j != jcur) {
+        jcur = j;
+        run = 0;
+        gcur = j == 0 ? g0 : (j == 1 ? g1 : (j == 2 ? g2 : g3));
       }
+      const uint32_t p = gcur + run++;
+      s.ckey[p] = to_key(pick16(v, b));
+      s.cidx[p] = static_cast<uint32_t>(jl + j * 128 + (b & 3));
     }
   }
   st.count += tot;
+  if (st.mode == kAcceptAll && st.count >= 2u * static_cast<uint32_t>(k)) {
+    // Seen at least 2k entries: fix an exact threshold early; fewer entries
+    // survive the filter afterwards than if the buffer were left to fill.
+    __syncthreads();
+    const uint32_t T = select_topk(s, 0, static_cast<int>(st.count), k, tid);
+    st.count = static_cast<uint32_t>(k);
+    set_exact_threshold(st, T);
+  }
 }
 
-// Stream one work item; on return the buffer holds min(k, #valid) winners of
-// the item in index order (exactly the item's top-k when it had >= k entries).
-__device__ __forceinline__ uint32_t stream_item(Smem& s, const Span& sp, int64_t c0, int64_t c1, int k, int& stage,
-                                                uint32_t& phase, int& par, int tid) {
+// Consumer side of the ring: g = stages consumed so far.
+__device__ __forceinline__ void load_stage(const Smem& s, uint32_t g, Lane16& v, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  const float* src = &s.ring[g % kStages][0];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float4 q = *reinterpret_cast<const float4*>(src + lane_offset(w, lane, j));
+    v.x[j][0] = q.x;
+    v.x[j][1] = q.y;
+    v.x[j][2] = q.z;
+    v.x[j][3] = q.w;
+  }
+}
+
+// Stream one work item through the ring. On return the buffer holds the
+// item's top min(k, #valid) entries in index order when the filter never
+// dropped a winner, which is always the case unless the starting mode was
+// kAtLeast; then the caller checks `count >= k` (see stream_row).
+__device__ __forceinline__ uint32_t stream_ring(Smem& s, const Span& sp, int64_t c0, int64_t c1, int k, uint32_t& g,
+                                                int& par, int mode0, float thr0, bool& compacted, int tid,
+                                                Producer* prod, const ItemSource* is) {
+  StreamState st;
+  st.count = 0;
+  st.mode = mode0;
+  st.thr = thr0;
+  st.par = par;
+  for (int t = 0; t < sp.nst; ++t) {
+    mbar_wait(&s.full[g % kStages], (g / kStages) & 1u);
+    Lane16 v;
+    load_stage(s, g, v, tid);
+    consume_values(s, st, v, &s.ring[g % kStages][0], sp.j0 + static_cast<int64_t>(t) * kStageElems, c0, c1, k, tid,
+                   prod, is);
+    ++g;
+  }
+  __syncthreads();  // the last stage's appends land before anyone reads the buffer
+  compacted = st.mode != mode0;
+  par = st.par;
+  return st.count;
+}
+
+// Same as stream_ring, reading the span straight from global memory (used to
+// redo a row whose speculative threshold turned out too high).
+__device__ __noinline__ uint32_t stream_global(Smem& s, const Span& sp, int64_t c0, int64_t c1, int k, int& par, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
   StreamState st;
   st.count = 0;
   st.mode = kAcceptAll;
   st.thr = 0.f;
   st.par = par;
   for (int t = 0; t < sp.nst; ++t) {
-    mbar_wait(&s.full[stage], phase);
-    consume_stage(s, st, stage, sp.j0 + static_cast<int64_t>(t) * kStageElems, c0, c1, k, tid);
-    if (++stage == kStages) {
-      stage = 0;
-      phase ^= 1u;
+    Lane16 v;
+    const uint64_t sbase = static_cast<uint64_t>(t) * kStageBytes;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint64_t off = sbase + 4u * static_cast<uint64_t>(lane_offset(w, lane, j));
+      float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (off + 16 <= sp.bytes) q = __ldg(reinterpret_cast<const float4*>(sp.src + off));
+      v.x[j][0] = q.x;
+      v.x[j][1] = q.y;
+      v.x[j][2] = q.z;
+      v.x[j][3] = q.w;
     }
+    consume_values(s, st, v, reinterpret_cast<const float*>(sp.src + sbase),
+                   sp.j0 + static_cast<int64_t>(t) * kStageElems, c0, c1, k, tid, nullptr, nullptr);
   }
-  bar_consumers();  // the last stage's appends land before anyone reads the buffer
-  if (st.count > static_cast<uint32_t>(k)) {
-    select_topk(s, 0, static_cast<int>(st.count), k, tid);
-    st.count = static_cast<uint32_t>(k);
-  }
+  __syncthreads();
   par = st.par;
   return st.count;
 }
 
 __device__ __forceinline__ void init_pipeline(Smem& s) {
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], kNumConsumerWarps);
-    }
+    for (int i = 0; i < kStages; ++i) mbar_init(&s.full[i], 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -676,38 +925,65 @@ __device__ __forceinline__ void init_pipeline(Smem& s) {
 
 // --------------------------------------------------------------- kernels
 // Many rows: one CTA per row, persistent over rows (row = blockIdx.x + i*gridDim.x).
-__global__ void __launch_bounds__(kThreads, 1)
+//
+// Rows after the first start from a lower estimate of their k-th value taken
+// from the row before (same CTA): the k-th value minus the gap between the
+// (3k/4)-th and k-th values. Entries >= the estimate are kept. If at least k
+// entries reach it, the k-th largest is >= the estimate, so every winner was
+// kept and the result is exact; otherwise the row is streamed again without an
+// estimate. Either way the output is the exact top-k.
+__global__ void __launch_bounds__(kThreads, kBlocksPerSM)
     topk_rows_kernel(const float* __restrict__ logits, int64_t row_stride, const int32_t* __restrict__ lengths,
                      int64_t num_rows, int k, int32_t* __restrict__ out) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>(smem_raw);
   init_pipeline(s);
   const int tid = threadIdx.x;
-  if (tid >= kConsumerThreads) {  // producer warp
-    if (tid == kConsumerThreads) {
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int64_t row = blockIdx.x; row < num_rows; row += gridDim.x) {
-        const int64_t L = clamp_len(lengths, row, row_stride);
-        produce_item(s, make_span(logits + row * row_stride, 0, L), stage, phase);
-      }
-    }
-    return;
+  const ItemSource is{logits, lengths, row_stride, num_rows, static_cast<int64_t>(gridDim.x), 0, -1};
+  Producer prod;
+  if (tid == 0) {
+    prod.row = blockIdx.x;
+    prod.g = 0;
+    producer_set_item(prod, is);
+    for (int i = 0; i < kStages; ++i) producer_issue(s, prod, is);
   }
-  int stage = 0, par = 0;
-  uint32_t phase = 0;
+  Producer* pp = tid == 0 ? &prod : nullptr;
+  uint32_t g = 0;
+  int par = 0;
+  bool have_est = false;
+  float est = 0.f;
   for (int64_t row = blockIdx.x; row < num_rows; row += gridDim.x) {
     const int64_t L = clamp_len(lengths, row, row_stride);
     const Span sp = make_span(logits + row * row_stride, 0, L);
-    const uint32_t m = stream_item(s, sp, 0, L, k, stage, phase, par, tid);
+    const bool spec = have_est && L > k;
+    bool compacted = false;
+    uint32_t m = stream_ring(s, sp, 0, L, k, g, par, spec ? kAtLeast : kAcceptAll, est, compacted, tid, pp, &is);
+    if (spec && !compacted && m < static_cast<uint32_t>(k)) {
+      m = stream_global(s, sp, 0, L, k, par, tid);  // estimate was too high
+      have_est = false;
+    }
+    if (m > static_cast<uint32_t>(k)) {
+      select_topk(s, 0, static_cast<int>(m), k, tid);
+      m = static_cast<uint32_t>(k);
+    }
     const int R = m ? sort_desc(s, 0, kMaxK, static_cast<int>(m), tid) : 0;
     write_row(s, R, static_cast<int>(m), k, out + row * static_cast<int64_t>(k), tid);
-    bar_consumers();  // outputs read cidx before the next row appends
+    if (m == static_cast<uint32_t>(k)) {
+      const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
+      const uint32_t kt = s.ckey[R + k - 1], ka = s.ckey[R + a];
+      const float vt = from_key(kt), va = from_key(ka);
+      const float e = vt - (va - vt);
+      have_est = kt != kNanKey && ka != kNanKey && isfinite(e);
+      est = e;
+    } else {
+      have_est = false;
+    }
+    __syncthreads();  // outputs and the estimate read the buffer before the next row appends
   }
 }
 
 // Few long rows: a cluster of CTAs per row (grid = num_rows * cluster size).
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kBlocksPerSM)
     topk_cluster_kernel(const float* __restrict__ logits, int64_t row_stride, const int32_t* __restrict__ lengths,
                         int64_t num_rows, int k, int32_t* __restrict__ out) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -726,23 +1002,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t c1 = min64(L, c0 + chunk);
   const float* row_ptr = logits + row * row_stride;
   const Span sp = make_span(row_ptr, c0, c1);
-  if (tid >= kConsumerThreads) {  // producer warp: issue, then leave the cluster barriers to consumers
-    if (tid == kConsumerThreads) {
-      int stage = 0;
-      uint32_t phase = 0;
-      produce_item(s, sp, stage, phase);
-    }
-    return;
-  }
   const int w = tid >> 5, lane = tid & 31;
-  int stage = 0, par = 0;
-  uint32_t phase = 0;
   const uint32_t m = static_cast<uint32_t>(min64(k, L));
   if (m == 0) {  // L == 0 for every rank alike: nothing streamed, no merge
     if (rank == 0) write_row(s, 0, 0, k, out + row * static_cast<int64_t>(k), tid);
     return;
   }
-  const uint32_t n_r = stream_item(s, sp, c0, c1, k, stage, phase, par, tid);
+  const ItemSource is{logits, lengths, row_stride, row + 1, 1, c0, c1};  // this one row only
+  Producer prod;
+  if (tid == 0) {
+    prod.row = row;
+    prod.g = 0;
+    producer_set_item(prod, is);
+    for (int i = 0; i < kStages; ++i) producer_issue(s, prod, is);
+  }
+  uint32_t g = 0;
+  int par = 0;
+  bool compacted = false;
+  uint32_t n_r = stream_ring(s, sp, c0, c1, k, g, par, kAcceptAll, 0.f, compacted, tid, tid == 0 ? &prod : nullptr,
+                             &is);
+  if (n_r > static_cast<uint32_t>(k)) {
+    select_topk(s, 0, static_cast<int>(n_r), k, tid);
+    n_r = static_cast<uint32_t>(k);
+  }
 
   // ---- merge phase 1: publish (count, min key, max key) of this rank
   const MinMax mm = block_minmax(s, 0, static_cast<int>(n_r), tid);
@@ -827,7 +1109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // exact: keep key > T plus a rank-ordered share of key == T; else keep key >= lo
   const uint32_t T = exact ? lo : lo - 1u;
   uint32_t g_r, q_r;
-  count_gt_eq(s, static_cast<int>(n_r), T, g_r, q_r, tid);
+  count_gt_eq(s, 0, static_cast<int>(n_r), T, g_r, q_r, tid);
   if (tid == 0) {
     s.pub[4] = g_r;
     s.pub[5] = exact ? q_r : 0u;
@@ -942,13 +1224,14 @@ static int device_setup(int dev, DeviceInfo* out) {
 static void plan(const DeviceInfo& d, int64_t num_rows, int64_t row_stride, int* cs_out, int64_t* grid_out) {
   constexpr int64_t kMinChunk = 16384;  // elements per rank worth a cluster merge
   int cs = 1;
-  if (num_rows < d.sms && d.max_cluster > 1) {
-    int64_t want = d.sms / (num_rows > 0 ? num_rows : 1);
+  const int64_t slots = static_cast<int64_t>(d.sms) * kBlocksPerSM;
+  if (num_rows < slots && d.max_cluster > 1) {
+    int64_t want = slots / (num_rows > 0 ? num_rows : 1);
     while (cs * 2 <= want && cs * 2 <= d.max_cluster && row_stride / (cs * 2) >= kMinChunk) cs *= 2;
   }
   *cs_out = cs;
   if (cs == 1)
-    *grid_out = num_rows < d.sms ? num_rows : d.sms;
+    *grid_out = num_rows < slots ? num_rows : slots;
   else
     *grid_out = num_rows * cs;
 }

@@ -34,8 +34,10 @@ full-size parity tests feed sampled rows to the oracle.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import hashlib
+import os
 from typing import Dict, Iterable, List, Optional
 
 import numpy as np
@@ -134,11 +136,12 @@ _LOG1P_CACHE: Dict[int, np.ndarray] = {}
 
 
 def _half_log1p(n: int) -> np.ndarray:
-    t = _LOG1P_CACHE.get(n)
-    if t is None:
-        t = 0.5 * np.log1p(np.arange(n, dtype=np.float64))
-        _LOG1P_CACHE[n] = t
-    return t
+    """0.5*log1p(d) for d = 0 .. n-1 (prefixes of one cached table)."""
+    t = _LOG1P_CACHE.get(0)
+    if t is None or len(t) < n:
+        t = 0.5 * np.log1p(np.arange(max(n, 131072), dtype=np.float64))
+        _LOG1P_CACHE[0] = t
+    return t[:n]
 
 
 def _row_values(s: Spec, row: int, L: int) -> np.ndarray:
@@ -160,11 +163,14 @@ def _row_values(s: Spec, row: int, L: int) -> np.ndarray:
     raise KeyError(s.name)
 
 
-def make_rows(name: str, rows: Iterable[int], row_stride: Optional[int] = None) -> Workload:
+def make_rows(name: str, rows: Iterable[int], row_stride: Optional[int] = None,
+              threads: int = 0) -> Workload:
     """Regenerate only ``rows`` of a workload, laid out at ``row_stride``.
 
     ``row_stride`` defaults to the workload's own stride; any stride >= the
     longest selected row gives the same valid values (padding is +inf).
+    Rows have independent streams, so they are filled by a thread pool
+    (``threads`` <= 0: one per CPU); the result does not depend on it.
     """
     s = _SPECS[name]
     rows = [int(r) for r in rows]
@@ -173,9 +179,21 @@ def make_rows(name: str, rows: Iterable[int], row_stride: Optional[int] = None) 
     stride = s.row_stride if row_stride is None else int(row_stride)
     if len(rows) and stride < int(L.max()):
         raise ValueError("row_stride shorter than a selected row")
-    out = np.full((len(rows), stride), np.inf, dtype=np.float32)
-    for i, r in enumerate(rows):
-        out[i, : L[i]] = _row_values(s, r, int(L[i]))
+    out = np.empty((len(rows), stride), dtype=np.float32)
+    if s.name == "prefill":
+        _half_log1p(int(L.max()) if len(rows) else 1)  # fill the shared table once
+
+    def fill(i: int) -> None:
+        out[i, : L[i]] = _row_values(s, rows[i], int(L[i]))
+        out[i, L[i]:] = np.inf
+
+    nt = threads if threads > 0 else (os.cpu_count() or 1)
+    if nt <= 1 or len(rows) < 8:
+        for i in range(len(rows)):
+            fill(i)
+    else:
+        with concurrent.futures.ThreadPoolExecutor(max_workers=min(nt, 32)) as ex:
+            list(ex.map(fill, range(len(rows))))
     return Workload(name=name, logits=out, lengths=L, k=s.k)
 
 
