@@ -33,8 +33,9 @@ def nvcc() -> str:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    stale = not os.path.exists(LIB) or any(
-        os.path.getmtime(p) > os.path.getmtime(LIB) for p in (SRC, HDR))
+    csrc = os.path.dirname(SRC)
+    deps = [HDR] + [os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh", ".h"))]
+    stale = not os.path.exists(LIB) or any(os.path.getmtime(p) > os.path.getmtime(LIB) for p in deps)
     if force or stale:
         tmp = LIB + ".tmp%d" % os.getpid()
         cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + [

@@ -9,7 +9,7 @@
 //   * One producer warp streams a row (or a chunk of it) into a ring of
 //     shared-memory stages with cp.async.bulk (TMA bulk copies, no
 //     multicast) completing on mbarriers.
-//   * Sixteen consumer warps turn each fp32 into an order-preserving uint32
+//   * Consumer warps turn each fp32 into an order-preserving uint32
 //     key only when it can still matter: a running threshold T (the exact
 //     k-th largest key among the entries seen so far) filters the stream, and
 //     survivors are appended to a shared-memory candidate buffer in index
@@ -160,6 +160,32 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t pari
   const unsigned long long t0 = global_ns();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_status, kStatusWaitTimeout);
+      return false;
+    }
+  }
+}
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about hint_ns pass, instead of spinning on the barrier.
+__device__ __forceinline__ bool mbar_try_wait_hint(unsigned long long* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for waits that are often long (a role idling until another
+// catches up): sleeps in the barrier instead of spinning.
+__device__ __forceinline__ bool mbar_wait_sleep(unsigned long long* bar, uint32_t parity) {
+  if (mbar_try_wait_hint(bar, parity, 2000u)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
     if (global_ns() - t0 > kWaitLimitNs) {
       atomicOr(&g_status, kStatusWaitTimeout);
       return false;
@@ -924,64 +950,6 @@ __device__ __forceinline__ void init_pipeline(Smem& s) {
 }
 
 // --------------------------------------------------------------- kernels
-// Many rows: one CTA per row, persistent over rows (row = blockIdx.x + i*gridDim.x).
-//
-// Rows after the first start from a lower estimate of their k-th value taken
-// from the row before (same CTA): the k-th value minus the gap between the
-// (3k/4)-th and k-th values. Entries >= the estimate are kept. If at least k
-// entries reach it, the k-th largest is >= the estimate, so every winner was
-// kept and the result is exact; otherwise the row is streamed again without an
-// estimate. Either way the output is the exact top-k.
-__global__ void __launch_bounds__(kThreads, kBlocksPerSM)
-    topk_rows_kernel(const float* __restrict__ logits, int64_t row_stride, const int32_t* __restrict__ lengths,
-                     int64_t num_rows, int k, int32_t* __restrict__ out) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  Smem& s = *reinterpret_cast<Smem*>(smem_raw);
-  init_pipeline(s);
-  const int tid = threadIdx.x;
-  const ItemSource is{logits, lengths, row_stride, num_rows, static_cast<int64_t>(gridDim.x), 0, -1};
-  Producer prod;
-  if (tid == 0) {
-    prod.row = blockIdx.x;
-    prod.g = 0;
-    producer_set_item(prod, is);
-    for (int i = 0; i < kStages; ++i) producer_issue(s, prod, is);
-  }
-  Producer* pp = tid == 0 ? &prod : nullptr;
-  uint32_t g = 0;
-  int par = 0;
-  bool have_est = false;
-  float est = 0.f;
-  for (int64_t row = blockIdx.x; row < num_rows; row += gridDim.x) {
-    const int64_t L = clamp_len(lengths, row, row_stride);
-    const Span sp = make_span(logits + row * row_stride, 0, L);
-    const bool spec = have_est && L > k;
-    bool compacted = false;
-    uint32_t m = stream_ring(s, sp, 0, L, k, g, par, spec ? kAtLeast : kAcceptAll, est, compacted, tid, pp, &is);
-    if (spec && !compacted && m < static_cast<uint32_t>(k)) {
-      m = stream_global(s, sp, 0, L, k, par, tid);  // estimate was too high
-      have_est = false;
-    }
-    if (m > static_cast<uint32_t>(k)) {
-      select_topk(s, 0, static_cast<int>(m), k, tid);
-      m = static_cast<uint32_t>(k);
-    }
-    const int R = m ? sort_desc(s, 0, kMaxK, static_cast<int>(m), tid) : 0;
-    write_row(s, R, static_cast<int>(m), k, out + row * static_cast<int64_t>(k), tid);
-    if (m == static_cast<uint32_t>(k)) {
-      const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
-      const uint32_t kt = s.ckey[R + k - 1], ka = s.ckey[R + a];
-      const float vt = from_key(kt), va = from_key(ka);
-      const float e = vt - (va - vt);
-      have_est = kt != kNanKey && ka != kNanKey && isfinite(e);
-      est = e;
-    } else {
-      have_est = false;
-    }
-    __syncthreads();  // outputs and the estimate read the buffer before the next row appends
-  }
-}
-
 // Few long rows: a cluster of CTAs per row (grid = num_rows * cluster size).
 __global__ void __launch_bounds__(kThreads, kBlocksPerSM)
     topk_cluster_kernel(const float* __restrict__ logits, int64_t row_stride, const int32_t* __restrict__ lengths,
@@ -1159,6 +1127,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM)
   write_row(s, R, static_cast<int>(m), k, out + row * static_cast<int64_t>(k), tid);
 }
 
+#include "rows_path.cuh"
+
 // ------------------------------------------------------------------ host
 struct DeviceInfo {
   int sms = 0;
@@ -1182,7 +1152,8 @@ static int device_setup(int dev, DeviceInfo* out) {
     d.major = p.major;
     d.minor = p.minor;
     const int smem = static_cast<int>(sizeof(Smem));
-    if (cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+    if (cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sizeof(rows::Smem))) != cudaSuccess ||
         cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
             cudaSuccess) {
       cudaGetLastError();
@@ -1224,14 +1195,15 @@ static int device_setup(int dev, DeviceInfo* out) {
 static void plan(const DeviceInfo& d, int64_t num_rows, int64_t row_stride, int* cs_out, int64_t* grid_out) {
   constexpr int64_t kMinChunk = 16384;  // elements per rank worth a cluster merge
   int cs = 1;
-  const int64_t slots = static_cast<int64_t>(d.sms) * kBlocksPerSM;
-  if (num_rows < slots && d.max_cluster > 1) {
-    int64_t want = slots / (num_rows > 0 ? num_rows : 1);
+  const int64_t row_slots = d.sms;                                         // one many-row CTA per SM
+  const int64_t cluster_slots = static_cast<int64_t>(d.sms) * kBlocksPerSM;  // cluster CTAs per GPU
+  if (num_rows < row_slots && d.max_cluster > 1) {
+    int64_t want = cluster_slots / (num_rows > 0 ? num_rows : 1);
     while (cs * 2 <= want && cs * 2 <= d.max_cluster && row_stride / (cs * 2) >= kMinChunk) cs *= 2;
   }
   *cs_out = cs;
   if (cs == 1)
-    *grid_out = num_rows < slots ? num_rows : slots;
+    *grid_out = num_rows < row_slots ? num_rows : row_slots;
   else
     *grid_out = num_rows * cs;
 }
@@ -1275,6 +1247,8 @@ static int launch(const DeviceInfo& d, const float* logits, int64_t row_stride, 
   cfg.stream = stream;
   cudaError_t e;
   if (cs == 1) {
+    cfg.blockDim = dim3(rows::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = sizeof(rows::Smem);
     e = cudaLaunchKernelEx(&cfg, topk_rows_kernel, logits, row_stride, lengths, num_rows, static_cast<int>(k), out);
   } else {
     attr[0].id = cudaLaunchAttributeClusterDimension;
