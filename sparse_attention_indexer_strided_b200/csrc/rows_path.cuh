@@ -38,15 +38,16 @@ constexpr int kFinishWarps = 4;
 constexpr int kFinishThreads = kFinishWarps * 32;  // 128
 constexpr int kProducerWarp = kFilterWarps + kFinishWarps;
 constexpr int kThreads = (kProducerWarp + 1) * 32;  // 416
-constexpr int kStageElems = 4096;
-constexpr uint32_t kStageBytes = kStageElems * 4;  // 16 KB
-constexpr int kStages = 6;                         // 96 KB ring
-constexpr int kWarpElems = kStageElems / kFilterWarps;  // 512 per warp and stage
-constexpr int kVals = kWarpElems / 32;                  // 16 per lane: 4 float4 groups
+constexpr int kGroups = 8;                              // float4 groups per lane and stage
+constexpr int kVals = 4 * kGroups;                      // 32 values per lane and stage
+constexpr int kWarpElems = 32 * kVals;                  // 1024 per warp and stage
+constexpr int kStageElems = kFilterWarps * kWarpElems;  // 8192
+constexpr uint32_t kStageBytes = kStageElems * 4;       // 32 KB
+constexpr int kStages = 3;                              // 96 KB ring
 constexpr int kFiltCap = 8192;                          // candidate buffer entries
-constexpr int kTrigger = kFiltCap - kStageElems;        // compact when a stage could overflow
+constexpr int kTrigger = kFiltCap / 2;                  // compact after a stage that leaves more
 constexpr int kHandCap = 4096;                          // handed-over candidates, at most
-constexpr int kBuckets = 4096;
+constexpr int kBuckets = 4096;                          // finisher bucket counters (32 per thread)
 constexpr int kPerThread = kFiltCap / kFilterThreads;   // 32 entries per filter thread
 constexpr int kScanPer = kBuckets / kFinishThreads;     // 32 counters per finisher thread
 constexpr uint32_t kInfKey = 0xFF800000u;               // key of +inf
@@ -55,9 +56,11 @@ constexpr int kKeepLimit = 2560;                        // approximate compactio
 constexpr int kSmallBucket = 16;                        // finisher: largest bucket ranked by direct counting
 constexpr int kSortPasses = 3;                          // finisher: bucket count passes, at most
 
-static_assert(kVals == 16, "a lane holds 4 float4 groups per stage");
+static_assert(kVals <= 32, "a lane's survivors of one stage form a 32-bit mask");
+static_assert(kFiltCap - kTrigger >= kStageElems / 2, "half a stage fits after a compaction");
 static_assert(kHandCap >= kMaxK && kTrigger >= kMaxK, "buffers must hold k entries");
-static_assert(kBuckets == 1 << 12, "bucket index is the top 12 bits of the composite key");
+static_assert(kBuckets == kScanPer * kFinishThreads && kBuckets <= 4096 && kScanPer % 4 == 0,
+              "bucket counters split evenly over the finisher threads");
 
 struct __align__(128) Smem {
   float ring[kStages][kStageElems];
@@ -91,7 +94,15 @@ struct __align__(128) Smem {
 static_assert(sizeof(Smem) <= 232448, "shared memory budget of one CTA per SM");
 
 __device__ __forceinline__ void bar_filter() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-__device__ __forceinline__ void bar_finish() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+__device__ __forceinline__ void bar_finish() { asm volatile("bar.sync 2, %0;" ::"n"(kFinishThreads) : "memory"); }
+
+// Warp sum by shuffles (the per-stage path avoids redux.sync, whose
+// throughput is far lower than that of shuffles).
+__device__ __forceinline__ uint32_t warp_sum(uint32_t x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
+  return x;
+}
 
 // Smallest float threshold t with (!(x < t)) == (key(x) > T) for every non-NaN x.
 // T at or above +inf's key has no such float: +inf is returned, which also
@@ -128,50 +139,9 @@ __device__ __forceinline__ RowSpan row_span(const float* row, int64_t L) {
 
 // ------------------------------------------------------------ filter warps
 // Position of value j (0..15) of a lane inside its stage: float4 group j/4 at
-// warp*512 + (j/4)*128 + lane*4 (conflict-free 128-bit shared loads).
+// warp*kWarpElems + (j/4)*128 + lane*4 (conflict-free 128-bit shared loads).
 __device__ __forceinline__ int val_offset(int w, int lane, int j) {
   return w * kWarpElems + (j >> 2) * 128 + lane * 4 + (j & 3);
-}
-
-// Appends the survivors in `msk` (bit j: value j of this lane) at positions
-// cnt.. of the candidate buffer, any order. One filter barrier per stage: each
-// warp publishes its survivor count, then every warp knows where to write and
-// the new count. `src` is the stage (ring slot or global memory); survivors
-// are re-read from it. Returns the new count (the same in every thread).
-template <bool kRing>
-__device__ __forceinline__ uint32_t append_stage(Smem& s, const float* src, uint32_t msk, uint32_t idx0, uint32_t cnt,
-                                                 int par, int w, int lane) {
-  const uint32_t nf = __popc(msk);
-  const uint32_t wt = __reduce_add_sync(kFull, nf);
-  const uint32_t rounds = __reduce_max_sync(kFull, nf);
-  if (lane == 0) reinterpret_cast<uint32_t*>(&s.red[par][0])[w] = wt;
-  bar_filter();
-  const uint4 a = s.red[par][0], b = s.red[par][1];
-  const uint32_t r[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-  uint32_t before = 0, tot = 0;
-#pragma unroll
-  for (int i = 0; i < kFilterWarps; ++i) {
-    before += i < w ? r[i] : 0u;
-    tot += r[i];
-  }
-  uint32_t pos = cnt + before;
-  const uint32_t lt = lanemask_lt();
-  uint32_t rest = msk;
-  for (uint32_t it = 0; it < rounds; ++it) {
-    const bool act = rest != 0u;
-    const uint32_t bal = __ballot_sync(kFull, act);
-    if (act) {
-      const int j = __ffs(rest) - 1;
-      rest &= rest - 1u;
-      const int off = val_offset(w, lane, j);
-      const uint32_t p = pos + __popc(bal & lt);
-      const float x = kRing ? src[off] : __ldg(src + off);
-      s.fkey[p] = to_key(x);
-      s.fidx[p] = idx0 + static_cast<uint32_t>(off);
-    }
-    pos += __popc(bal);
-  }
-  return cnt + tot;
 }
 
 __device__ __forceinline__ uint32_t pass_mask(const float (&v)[kVals], float t) {
@@ -463,59 +433,83 @@ __device__ __forceinline__ void compact_any(Smem& s, Filter& f, int m, int tid) 
   f.compacted = true;
 }
 
-// One stage of 4096 values, synchronous form (one filter barrier per stage):
-// src is the stage's first float in global memory, sj0 its row index; edge:
-// the stage may hold indices outside [0, L); avail: readable bytes.
-__device__ __forceinline__ void filter_stage_global(Smem& s, Filter& f, const float* src, int64_t sj0, int64_t L,
-                                                    bool edge, uint32_t avail, int m, int tid) {
+// Writes this warp's survivors (bit j of msk: value j of the lane; values
+// re-read from src, the stage in the ring or in global memory) at positions
+// pos.., one survivor per lane and round.
+template <bool kRing>
+__device__ __forceinline__ void put_survivors(Smem& s, const float* src, uint32_t msk, uint32_t idx0, uint32_t pos,
+                                              int w, int lane) {
+  const uint32_t lt = lanemask_lt();
+  uint32_t rest = msk;
+  for (;;) {
+    const bool act = rest != 0u;
+    const uint32_t bal = __ballot_sync(kFull, act);
+    if (bal == 0u) break;
+    if (act) {
+      const int j = __ffs(rest) - 1;
+      rest &= rest - 1u;
+      const int off = val_offset(w, lane, j);
+      const uint32_t p = pos + __popc(bal & lt);
+      const float x = kRing ? src[off] : __ldg(src + off);
+      s.fkey[p] = to_key(x);
+      s.fidx[p] = idx0 + static_cast<uint32_t>(off);
+    }
+    pos += __popc(bal);
+  }
+}
+
+// A stage whose survivors do not fit behind the buffer's contents (rare: no
+// usable threshold yet, or values rising along the row): the warps write in
+// two halves of four, compacting first whenever a half would not fit. A half
+// with more than the free space implies more than kTrigger >= m entries held,
+// so the compaction applies; afterwards a half (<= kStageElems / 2) fits. Masks
+// taken before a compaction are supersets of the current ones, which is
+// harmless: the final ranking is exact.
+template <bool kRing>
+__device__ __noinline__ void take_stage_split(Smem& s, Filter& f, uint4 ra, uint4 rb, const float* src, uint32_t msk,
+                                              uint32_t idx0, int m, int tid) {
   const int w = tid >> 5, lane = tid & 31;
-  float v[kVals];
+  const uint32_t r[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+  for (int half = 0; half < 2; ++half) {
+    uint32_t tot = 0, before = 0;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int off = w * kWarpElems + q * 128 + lane * 4;
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (4u * static_cast<uint32_t>(off) + 16u <= avail) x = __ldg(reinterpret_cast<const float4*>(src + off));
-    v[4 * q + 0] = x.x;
-    v[4 * q + 1] = x.y;
-    v[4 * q + 2] = x.z;
-    v[4 * q + 3] = x.w;
+    for (int i = 0; i < 4; ++i) {
+      const int ww = 4 * half + i;
+      tot += r[ww];
+      before += ww < w ? r[ww] : 0u;
+    }
+    if (f.cnt + tot > static_cast<uint32_t>(kFiltCap)) compact_any(s, f, m, tid);
+    if ((w >> 2) == half) put_survivors<kRing>(s, src, msk, idx0, f.cnt + before, w, lane);
+    f.cnt += tot;
+    bar_filter();  // this half's entries are visible to a following compaction
   }
-  uint32_t msk = pass_mask(v, f.t);
-  if (edge) {
-    int lo, hi;
-    stage_bounds(sj0, L, lo, hi);
-    msk &= range_mask(w, lane, lo, hi);
-  }
-  f.cnt = append_stage<false>(s, src, msk, static_cast<uint32_t>(sj0), f.cnt, f.par, w, lane);
-  f.par ^= 1;
-  if (f.cnt > static_cast<uint32_t>(kTrigger)) compact_any(s, f, m, tid);
 }
 
-// The speculative threshold let fewer than m values through: stream the row
-// again from global memory with no threshold.
-__device__ __noinline__ void refilter_from_global(Smem& s, Filter& f, const RowSpan& sp, int64_t L, int m, int tid) {
-  f.cnt = 0;
-  f.t = __int_as_float(0xff800000);  // -inf: keep everything
-  f.compacted = false;
-  for (int st = 0; st < sp.nst; ++st) {
-    const float* src = reinterpret_cast<const float*>(sp.src + static_cast<uint64_t>(st) * kStageBytes);
-    const uint32_t avail = st + 1 == sp.nst ? sp.last_bytes : kStageBytes;
-    filter_stage_global(s, f, src, sp.j0 + static_cast<int64_t>(st) * kStageElems, L, st == 0 || st + 1 == sp.nst,
-                        avail, m, tid);
+// Takes one stage after the filter barrier that completed its per-warp counts.
+template <bool kRing>
+__device__ __forceinline__ void take_stage(Smem& s, Filter& f, const uint4* red, const float* src, uint32_t msk,
+                                           uint32_t idx0, int m, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  const uint4 ra = red[0], rb = red[1];
+  const uint32_t r[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+  uint32_t before = 0, tot = 0;
+#pragma unroll
+  for (int i = 0; i < kFilterWarps; ++i) {
+    before += i < w ? r[i] : 0u;
+    tot += r[i];
   }
-  bar_filter();
+  if (f.cnt + tot <= static_cast<uint32_t>(kFiltCap)) {
+    put_survivors<kRing>(s, src, msk, idx0, f.cnt + before, w, lane);
+    f.cnt += tot;
+  } else {
+    take_stage_split<kRing>(s, f, ra, rb, src, msk, idx0, m, tid);
+  }
 }
 
-// ---- ring path
-__device__ __forceinline__ void load_slot(const Smem& s, int slot, int w, int lane, float (&v)[kVals]) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float4 x = *reinterpret_cast<const float4*>(&s.ring[slot][w * kWarpElems + q * 128 + lane * 4]);
-    v[4 * q + 0] = x.x;
-    v[4 * q + 1] = x.y;
-    v[4 * q + 2] = x.z;
-    v[4 * q + 3] = x.w;
-  }
+// Publishes this warp's survivor count (read after the next filter barrier).
+__device__ __forceinline__ void publish(uint4* red, uint32_t msk, int w, int lane) {
+  const uint32_t wt = __reduce_add_sync(kFull, __popc(msk));
+  if (lane == 0) reinterpret_cast<uint32_t*>(red)[w] = wt;
 }
 
 __device__ __forceinline__ uint32_t stage_mask(const float (&v)[kVals], float t, bool edge, int64_t sj0, int64_t L,
@@ -529,44 +523,47 @@ __device__ __forceinline__ uint32_t stage_mask(const float (&v)[kVals], float t,
   return msk;
 }
 
-// Publishes this warp's survivor count of stage g (read after the next filter
-// barrier).
-__device__ __forceinline__ void publish(Smem& s, uint32_t msk, uint32_t g, int w, int lane) {
-  const uint32_t wt = __reduce_add_sync(kFull, __popc(msk));
-  if (lane == 0) reinterpret_cast<uint32_t*>(&s.red[g & 1u][0])[w] = wt;
+// The speculative threshold let fewer than m values through: stream the row
+// again from global memory with no threshold (one filter barrier per stage).
+__device__ __noinline__ void refilter_from_global(Smem& s, Filter& f, const RowSpan& sp, int64_t L, int m, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  f.cnt = 0;
+  f.t = __int_as_float(0xff800000);  // -inf: keep everything
+  f.compacted = false;
+  for (int st = 0; st < sp.nst; ++st) {
+    const float* src = reinterpret_cast<const float*>(sp.src + static_cast<uint64_t>(st) * kStageBytes);
+    const uint32_t avail = st + 1 == sp.nst ? sp.last_bytes : kStageBytes;
+    const int64_t sj0 = sp.j0 + static_cast<int64_t>(st) * kStageElems;
+    float v[kVals];
+#pragma unroll
+    for (int q = 0; q < kGroups; ++q) {
+      const int off = w * kWarpElems + q * 128 + lane * 4;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (4u * static_cast<uint32_t>(off) + 16u <= avail) x = __ldg(reinterpret_cast<const float4*>(src + off));
+      v[4 * q + 0] = x.x;
+      v[4 * q + 1] = x.y;
+      v[4 * q + 2] = x.z;
+      v[4 * q + 3] = x.w;
+    }
+    const uint32_t msk = stage_mask(v, f.t, st == 0 || st + 1 == sp.nst, sj0, L, w, lane);
+    publish(&s.red[f.par][0], msk, w, lane);
+    bar_filter();
+    take_stage<false>(s, f, &s.red[f.par][0], src, msk, static_cast<uint32_t>(sj0), m, tid);
+    f.par ^= 1;
+    if (f.cnt > static_cast<uint32_t>(kTrigger)) compact_any(s, f, m, tid);
+  }
+  bar_filter();
 }
 
-// Writes this warp's survivors of stage g (re-read from the ring slot) behind
-// those of the warps before it, from the counts every warp published for
-// stage g before the last filter barrier. Returns the new count (uniform).
-__device__ __forceinline__ uint32_t write_stage(Smem& s, const float* slot, uint32_t msk, uint32_t idx0, uint32_t cnt,
-                                                uint32_t g, int w, int lane) {
-  const uint32_t rounds = __reduce_max_sync(kFull, __popc(msk));
-  const uint4 a = s.red[g & 1u][0], b = s.red[g & 1u][1];
-  const uint32_t r[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-  uint32_t before = 0, tot = 0;
+__device__ __forceinline__ void load_slot(const Smem& s, int slot, int w, int lane, float (&v)[kVals]) {
 #pragma unroll
-  for (int i = 0; i < kFilterWarps; ++i) {
-    before += i < w ? r[i] : 0u;
-    tot += r[i];
+  for (int q = 0; q < kGroups; ++q) {
+    const float4 x = *reinterpret_cast<const float4*>(&s.ring[slot][w * kWarpElems + q * 128 + lane * 4]);
+    v[4 * q + 0] = x.x;
+    v[4 * q + 1] = x.y;
+    v[4 * q + 2] = x.z;
+    v[4 * q + 3] = x.w;
   }
-  uint32_t pos = cnt + before;
-  const uint32_t lt = lanemask_lt();
-  uint32_t rest = msk;
-  for (uint32_t it = 0; it < rounds; ++it) {
-    const bool act = rest != 0u;
-    const uint32_t bal = __ballot_sync(kFull, act);
-    if (act) {
-      const int j = __ffs(rest) - 1;
-      rest &= rest - 1u;
-      const int off = val_offset(w, lane, j);
-      const uint32_t p = pos + __popc(bal & lt);
-      s.fkey[p] = to_key(slot[off]);
-      s.fidx[p] = idx0 + static_cast<uint32_t>(off);
-    }
-    pos += __popc(bal);
-  }
-  return cnt + tot;
 }
 
 __device__ void filter_loop(Smem& s, const float* logits, int64_t row_stride, const int32_t* lengths,
@@ -597,46 +594,19 @@ __device__ void filter_loop(Smem& s, const float* logits, int64_t row_stride, co
     }
     f.cnt = 0;
     f.compacted = false;
-    if (sp.nst > 0) {
-      // Software pipeline, one filter barrier per stage: in the iteration of
-      // stage g the warps publish the survivor counts of stage g+1 (values
-      // loaded one iteration earlier) and write the survivors of stage g,
-      // while the values of stage g+2 are being loaded.
-      uint32_t msk;  // survivors of stage g
-      float vn[kVals];
-      {
-        const int slot = static_cast<int>(g % kStages);
-        mbar_wait(&s.full[slot], (g / kStages) & 1u);
-        load_slot(s, slot, w, lane, vn);
-        msk = stage_mask(vn, f.t, true, sp.j0, L, w, lane);
-        publish(s, msk, g, w, lane);
-        if (sp.nst > 1) {
-          const int ns = static_cast<int>((g + 1) % kStages);
-          mbar_wait(&s.full[ns], ((g + 1) / kStages) & 1u);
-          load_slot(s, ns, w, lane, vn);
-        }
-      }
-      for (int st = 0; st < sp.nst; ++st, ++g) {
-        bar_filter();  // counts of stage g are complete
-        uint32_t msk_next = 0;
-        if (st + 1 < sp.nst) {
-          const int64_t sj = sp.j0 + static_cast<int64_t>(st + 1) * kStageElems;
-          msk_next = stage_mask(vn, f.t, st + 2 == sp.nst, sj, L, w, lane);
-          publish(s, msk_next, g + 1, w, lane);
-        }
-        const int slot = static_cast<int>(g % kStages);
-        f.cnt = write_stage(s, &s.ring[slot][0], msk,
-                            static_cast<uint32_t>(sp.j0 + static_cast<int64_t>(st) * kStageElems), f.cnt, g, w, lane);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.empty[slot]);
-        if (st + 2 < sp.nst) {
-          const int ns = static_cast<int>((g + 2) % kStages);
-          mbar_wait(&s.full[ns], ((g + 2) / kStages) & 1u);
-          load_slot(s, ns, w, lane, vn);
-        }
-        msk = msk_next;
-        if (f.cnt > static_cast<uint32_t>(kTrigger)) compact_any(s, f, m, tid);
-      }
+    for (int st = 0; st < sp.nst; ++st, ++g) {
+      const int slot = static_cast<int>(g % kStages);
+      const int64_t sj0 = sp.j0 + static_cast<int64_t>(st) * kStageElems;
+      mbar_wait(&s.full[slot], (g / kStages) & 1u);
+      float v[kVals];
+      load_slot(s, slot, w, lane, v);
+      const uint32_t msk = stage_mask(v, f.t, st == 0 || st + 1 == sp.nst, sj0, L, w, lane);
+      publish(&s.red[g & 1u][0], msk, w, lane);
+      bar_filter();  // every warp's count of this stage is published
+      take_stage<true>(s, f, &s.red[g & 1u][0], &s.ring[slot][0], msk, static_cast<uint32_t>(sj0), m, tid);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.empty[slot]);
+      if (f.cnt > static_cast<uint32_t>(kTrigger)) compact_any(s, f, m, tid);
     }
     bar_filter();  // every append is visible
     if (spec && !f.compacted && f.cnt < static_cast<uint32_t>(m)) refilter_from_global(s, f, sp, L, m, tid);
@@ -673,7 +643,9 @@ __device__ void filter_loop(Smem& s, const float* logits, int64_t row_stride, co
 // bucket's start plus the number of bucket members ahead of it.
 __device__ __forceinline__ int bucket_shift(uint64_t cmax) {
   const int bits = cmax ? 64 - __clzll(static_cast<long long>(cmax)) : 0;
-  return bits > 12 ? bits - 12 : 0;
+  int sh = bits > 12 ? bits - 12 : 0;  // cmax >> sh < 4096
+  if ((cmax >> sh) >= static_cast<uint64_t>(kBuckets)) ++sh;
+  return sh;
 }
 
 __device__ void finish_one(Smem& s, int k, int32_t* __restrict__ out, int h, int fid) {
@@ -699,9 +671,12 @@ __device__ void finish_one(Smem& s, int k, int32_t* __restrict__ out, int h, int
       s.nred[2][fw] = imax;
     }
     bar_finish();
-    kmin = min(min(s.nred[0][0], s.nred[0][1]), min(s.nred[0][2], s.nred[0][3]));
-    kmax = max(max(s.nred[1][0], s.nred[1][1]), max(s.nred[1][2], s.nred[1][3]));
-    imax = max(max(s.nred[2][0], s.nred[2][1]), max(s.nred[2][2], s.nred[2][3]));
+#pragma unroll
+    for (int ww = 0; ww < kFinishWarps; ++ww) {
+      kmin = min(kmin, s.nred[0][ww]);
+      kmax = max(kmax, s.nred[1][ww]);
+      imax = max(imax, s.nred[2][ww]);
+    }
     uint64_t cmax = (static_cast<uint64_t>(kmax - kmin) << 32) | imax;
     int sh = bucket_shift(cmax);
     auto comp = [&](uint32_t key, uint32_t idx) -> uint64_t {
@@ -769,7 +744,8 @@ __device__ void finish_one(Smem& s, int k, int32_t* __restrict__ out, int h, int
       big = __reduce_max_sync(kFull, big);
       if (lane == 0) s.nred[4][fw] = big;
       bar_finish();
-      big = max(max(s.nred[4][0], s.nred[4][1]), max(s.nred[4][2], s.nred[4][3]));
+#pragma unroll
+      for (int ww = 0; ww < kFinishWarps; ++ww) big = max(big, s.nred[4][ww]);
       if (big <= static_cast<uint32_t>(kSmallBucket) || sh == 0 || pass == kSortPasses - 1) break;
       cmax = ((static_cast<uint64_t>(bm) + 1u) << sh) - 1u;
       sh = bucket_shift(cmax);
@@ -810,7 +786,7 @@ __device__ void finish_one(Smem& s, int k, int32_t* __restrict__ out, int h, int
     if (n > 0 && m == k) {
       const uint32_t kt = s.rec[0], ka = s.rec[1];
       const float vt = from_key(kt), va = from_key(ka);
-      e = vt - (va - vt);
+      e = vt - 0.5f * (va - vt);
       ok = kt != kNanKey && ka != kNanKey && isfinite(e);
     }
     s.est[h & 1] = e;
