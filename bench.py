@@ -78,8 +78,14 @@ def load_peaks():
 
 
 def source_sha():
-    src = os.path.join(ROOT, "sparse_attention_indexer_strided_b200", "csrc", "dsa_topk.cu")
-    return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    """Digest of every kernel source file (a traffic figure is only valid for it)."""
+    csrc = os.path.join(ROOT, "sparse_attention_indexer_strided_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def profiled_traffic(config):

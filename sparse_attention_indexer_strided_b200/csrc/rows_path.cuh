@@ -53,6 +53,8 @@ constexpr int kScanPer = kBuckets / kFinishThreads;     // 32 counters per finis
 constexpr uint32_t kInfKey = 0xFF800000u;               // key of +inf
 constexpr int kRounds = 4;                              // radix rounds of 8 bits
 constexpr int kKeepLimit = 2560;                        // approximate compaction keeps at most this many
+constexpr int kSampleChunks = kFilterWarps * kGroups;   // runs of 128 sampled for a row's first threshold
+constexpr int64_t kSampleMinLen = 4 * kStageElems;      // shorter rows start with no threshold
 constexpr int kSmallBucket = 16;                        // finisher: largest bucket ranked by direct counting
 constexpr int kSortPasses = 3;                          // finisher: bucket count passes, at most
 
@@ -414,8 +416,20 @@ struct Filter {
   float t;            // keep x unless x < t
   int par;            // stage parity of s.red on the synchronous path
   bool compacted;     // the row was compacted at least once
+  bool strict;        // t already excludes values equal to the held m-th key
   uint32_t last_key;  // the last compaction kept every key >= last_key, at least m of them
 };
+
+// Holding at least m candidates, every one at or above the threshold t: a
+// later value equal to t has a larger index than all of them and cannot enter
+// the top m, so the threshold becomes strict (rows of tied values then stop
+// filling the buffer).
+__device__ __forceinline__ void tighten(Filter& f, int m) {
+  if (!f.strict && m > 0 && f.cnt >= static_cast<uint32_t>(m)) {
+    f.t = above(to_key(f.t));
+    f.strict = true;
+  }
+}
 
 // Bounds the buffer again: the approximate pass, else the exact one.
 __device__ __forceinline__ void compact_any(Smem& s, Filter& f, int m, int tid) {
@@ -424,11 +438,14 @@ __device__ __forceinline__ void compact_any(Smem& s, Filter& f, int m, int tid) 
     f.cnt = kept;
     f.t = lo > kInfKey ? __int_as_float(0x7f800000) : from_key(lo);
     f.last_key = lo;
+    f.strict = false;
+    tighten(f, m);
   } else {
     const uint32_t T = compact_exact(s, static_cast<int>(f.cnt), m, tid);
     f.cnt = static_cast<uint32_t>(m);
     f.t = above(T);
     f.last_key = T;
+    f.strict = true;
   }
   f.compacted = true;
 }
@@ -530,6 +547,7 @@ __device__ __noinline__ void refilter_from_global(Smem& s, Filter& f, const RowS
   f.cnt = 0;
   f.t = __int_as_float(0xff800000);  // -inf: keep everything
   f.compacted = false;
+  f.strict = false;
   for (int st = 0; st < sp.nst; ++st) {
     const float* src = reinterpret_cast<const float*>(sp.src + static_cast<uint64_t>(st) * kStageBytes);
     const uint32_t avail = st + 1 == sp.nst ? sp.last_bytes : kStageBytes;
@@ -551,8 +569,38 @@ __device__ __noinline__ void refilter_from_global(Smem& s, Filter& f, const RowS
     take_stage<false>(s, f, &s.red[f.par][0], src, msk, static_cast<uint32_t>(sj0), m, tid);
     f.par ^= 1;
     if (f.cnt > static_cast<uint32_t>(kTrigger)) compact_any(s, f, m, tid);
+    tighten(f, m);
   }
   bar_filter();
+}
+
+// A threshold for a row with no estimate, from a sample of kStageElems values
+// in kSampleChunks evenly spaced runs of 128 (aligned 16-byte blocks inside
+// the row): the value with as many sampled values above it as 1.5 times the
+// share of m in the sample, plus 16. Returns -inf when the sample gives none.
+__device__ __noinline__ float sample_threshold(Smem& s, const float* row, int64_t L, int m, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(row);
+  const uintptr_t as = a & ~static_cast<uintptr_t>(15);
+  const int64_t j0 = -static_cast<int64_t>((a - as) >> 2);  // row index of the aligned base
+  const int64_t span = L - j0;                               // floats from the aligned base to the row end
+#pragma unroll
+  for (int q = 0; q < kGroups; ++q) {
+    const int64_t c = w * kGroups + q;
+    const int64_t b = ((span - 128) * c / (kSampleChunks - 1)) & ~static_cast<int64_t>(3);
+    const float4 x = __ldg(reinterpret_cast<const float4*>(as) + (b >> 2) + lane);
+    const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t j = j0 + b + 4 * lane + i;
+      s.fkey[val_offset(w, lane, 4 * q + i)] = (j >= 0 && j < L) ? to_key(xv[i]) : 0u;  // 0: below every key
+    }
+  }
+  bar_filter();
+  const double share = static_cast<double>(kStageElems) * m / static_cast<double>(L);
+  const uint32_t need = min(static_cast<uint32_t>(kStageElems - 8), static_cast<uint32_t>(1.5 * share) + 16u);
+  const uint32_t T = filter_kth(s, kStageElems, need, FKey{&s}, FAll{}, tid);
+  return (T == 0u || T >= kInfKey) ? __int_as_float(0xff800000) : from_key(T);
 }
 
 __device__ __forceinline__ void load_slot(const Smem& s, int slot, int w, int lane, float (&v)[kVals]) {
@@ -592,8 +640,16 @@ __device__ void filter_loop(Smem& s, const float* logits, int64_t row_stride, co
         f.t = s.own_key > kInfKey ? __int_as_float(0x7f800000) : from_key(s.own_key);
       }
     }
+    if (m == k && !spec && L >= kSampleMinLen) {
+      const float ts = sample_threshold(s, logits + row * row_stride, L, m, tid);
+      if (ts > __int_as_float(0xff800000)) {
+        spec = true;
+        f.t = ts;
+      }
+    }
     f.cnt = 0;
     f.compacted = false;
+    f.strict = false;
     for (int st = 0; st < sp.nst; ++st, ++g) {
       const int slot = static_cast<int>(g % kStages);
       const int64_t sj0 = sp.j0 + static_cast<int64_t>(st) * kStageElems;
@@ -607,6 +663,7 @@ __device__ void filter_loop(Smem& s, const float* logits, int64_t row_stride, co
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.empty[slot]);
       if (f.cnt > static_cast<uint32_t>(kTrigger)) compact_any(s, f, m, tid);
+      tighten(f, m);
     }
     bar_filter();  // every append is visible
     if (spec && !f.compacted && f.cnt < static_cast<uint32_t>(m)) refilter_from_global(s, f, sp, L, m, tid);
