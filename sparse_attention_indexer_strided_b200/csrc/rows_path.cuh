@@ -55,6 +55,7 @@ constexpr int kRounds = 4;                              // radix rounds of 8 bit
 constexpr int kKeepLimit = 2560;                        // approximate compaction keeps at most this many
 constexpr int kSampleChunks = kFilterWarps * kGroups;   // runs of 128 sampled for a row's first threshold
 constexpr int64_t kSampleMinLen = 4 * kStageElems;      // shorter rows start with no threshold
+constexpr int kBigBucket = 64;                          // finisher: larger buckets are sorted instead
 constexpr int kSmallBucket = 16;                        // finisher: largest bucket ranked by direct counting
 constexpr int kSortPasses = 3;                          // finisher: bucket count passes, at most
 
@@ -617,7 +618,9 @@ __device__ __forceinline__ void load_slot(const Smem& s, int slot, int w, int la
 __device__ void filter_loop(Smem& s, const float* logits, int64_t row_stride, const int32_t* lengths,
                             int64_t num_rows, int k, int tid) {
   const int w = tid >> 5, lane = tid & 31;
-  uint32_t g = 0;  // ring stages consumed
+  int slot = 0;         // ring slot of the next stage
+  uint32_t phase = 0u;  // its full-barrier phase parity
+  uint32_t par = 0u;    // parity of the per-stage counts in s.red
   Filter f;
   f.par = 0;
   int h = 0;
@@ -650,20 +653,24 @@ __device__ void filter_loop(Smem& s, const float* logits, int64_t row_stride, co
     f.cnt = 0;
     f.compacted = false;
     f.strict = false;
-    for (int st = 0; st < sp.nst; ++st, ++g) {
-      const int slot = static_cast<int>(g % kStages);
-      const int64_t sj0 = sp.j0 + static_cast<int64_t>(st) * kStageElems;
-      mbar_wait(&s.full[slot], (g / kStages) & 1u);
+    int32_t sj0 = static_cast<int32_t>(sp.j0);  // row index of the stage's first float (< L <= INT32_MAX)
+    for (int st = 0; st < sp.nst; ++st, sj0 += kStageElems) {
+      mbar_wait(&s.full[slot], phase);
       float v[kVals];
       load_slot(s, slot, w, lane, v);
       const uint32_t msk = stage_mask(v, f.t, st == 0 || st + 1 == sp.nst, sj0, L, w, lane);
-      publish(&s.red[g & 1u][0], msk, w, lane);
+      publish(&s.red[par][0], msk, w, lane);
       bar_filter();  // every warp's count of this stage is published
-      take_stage<true>(s, f, &s.red[g & 1u][0], &s.ring[slot][0], msk, static_cast<uint32_t>(sj0), m, tid);
+      take_stage<true>(s, f, &s.red[par][0], &s.ring[slot][0], msk, static_cast<uint32_t>(sj0), m, tid);
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.empty[slot]);
       if (f.cnt > static_cast<uint32_t>(kTrigger)) compact_any(s, f, m, tid);
       tighten(f, m);
+      par ^= 1u;
+      if (++slot == kStages) {
+        slot = 0;
+        phase ^= 1u;
+      }
     }
     bar_filter();  // every append is visible
     if (spec && !f.compacted && f.cnt < static_cast<uint32_t>(m)) refilter_from_global(s, f, sp, L, m, tid);
@@ -705,6 +712,43 @@ __device__ __forceinline__ int bucket_shift(uint64_t cmax) {
   return sh;
 }
 
+// Candidates [0, n) ordered in place by (key descending, index ascending) with
+// a bitonic network over the next power of two (padding keys 0 sort last),
+// then the first m indices written. Ends with a finisher barrier.
+__device__ __noinline__ void finish_sorted(Smem& s, int n, int m, int k, int32_t* __restrict__ o, int fid) {
+  int N = 1;
+  while (N < n) N <<= 1;
+  for (int e = n + fid; e < N; e += kFinishThreads) {
+    s.hkey[e] = 0u;
+    s.hidx[e] = 0xFFFFFFFFu;
+  }
+  bar_finish();
+  for (int size = 2; size <= N; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = fid; t < (N >> 1); t += kFinishThreads) {
+        const int i = 2 * t - (t & (stride - 1));
+        const int j = i + stride;
+        const uint32_t ki = s.hkey[i], ii = s.hidx[i], kj = s.hkey[j], ij = s.hidx[j];
+        const bool j_first = kj > ki || (kj == ki && ij < ii);  // j belongs before i
+        if (j_first == ((i & size) == 0)) {
+          s.hkey[i] = kj;
+          s.hidx[i] = ij;
+          s.hkey[j] = ki;
+          s.hidx[j] = ii;
+        }
+      }
+      bar_finish();
+    }
+  }
+  const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
+  for (int p = fid; p < m; p += kFinishThreads) {
+    o[p] = static_cast<int32_t>(s.hidx[p]);
+    if (p == k - 1) s.rec[0] = s.hkey[p];
+    if (p == a) s.rec[1] = s.hkey[p];
+  }
+  bar_finish();
+}
+
 __device__ void finish_one(Smem& s, int k, int32_t* __restrict__ out, int h, int fid) {
   const int fw = fid >> 5, lane = fid & 31;
   const int n = s.h_n, m = s.h_m;
@@ -741,6 +785,7 @@ __device__ void finish_one(Smem& s, int k, int32_t* __restrict__ out, int h, int
     };
     uint4* bc4 = reinterpret_cast<uint4*>(&s.bcnt[fid * kScanPer]);
     const uint32_t mm1 = static_cast<uint32_t>(m - 1);
+    uint32_t big = 0;
     for (int pass = 0;; ++pass) {
 #pragma unroll
       for (int i = 0; i < kScanPer / 4; ++i) bc4[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -794,7 +839,7 @@ __device__ void finish_one(Smem& s, int k, int32_t* __restrict__ out, int h, int
       }
       bar_finish();
       const uint32_t bm = s.bc[4];
-      uint32_t big = 0;  // largest bucket at or before bm
+      big = 0;  // largest bucket at or before bm
 #pragma unroll
       for (int i = 0; i < kScanPer; ++i)
         if (static_cast<uint32_t>(fid * kScanPer + i) <= bm) big = max(big, c[i]);
@@ -808,34 +853,40 @@ __device__ void finish_one(Smem& s, int k, int32_t* __restrict__ out, int h, int
       sh = bucket_shift(cmax);
       bar_finish();  // bc[4] and nred[4] are rewritten by the next pass
     }
-    for (int e = fid; e < n; e += kFinishThreads) {
-      const uint64_t cc = comp(s.hkey[e], s.hidx[e]);
-      if (cc > cmax) continue;
-      const uint32_t p = atomicAdd(&s.bcnt[static_cast<uint32_t>(cc >> sh)], 1u);
-      s.perm[p] = static_cast<uint16_t>(e);
-    }
-    bar_finish();  // bcnt[b] is now the end of bucket b (= start of b + 1)
-    const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
-    for (int e = fid; e < n; e += kFinishThreads) {
-      const uint32_t key = s.hkey[e], idx = s.hidx[e];
-      const uint64_t cc = comp(key, idx);
-      if (cc > cmax) continue;
-      const uint32_t b = static_cast<uint32_t>(cc >> sh);
-      const uint32_t s0 = b ? s.bcnt[b - 1] : 0u, s1 = s.bcnt[b];
-      if (s0 >= static_cast<uint32_t>(m)) continue;
-      uint32_t r = s0;
-      for (uint32_t q = s0; q < s1; ++q) {
-        const uint32_t j = s.perm[q];
-        const uint32_t kj = s.hkey[j], ij = s.hidx[j];
-        r += kj > key || (kj == key && ij < idx);
+    if (big > static_cast<uint32_t>(kBigBucket)) {
+      // many candidates share a bucket (values on a coarse grid): counting
+      // ranks inside it would be quadratic, so sort everything instead
+      finish_sorted(s, n, m, k, o, fid);
+    } else {
+      for (int e = fid; e < n; e += kFinishThreads) {
+        const uint64_t cc = comp(s.hkey[e], s.hidx[e]);
+        if (cc > cmax) continue;
+        const uint32_t p = atomicAdd(&s.bcnt[static_cast<uint32_t>(cc >> sh)], 1u);
+        s.perm[p] = static_cast<uint16_t>(e);
       }
-      if (r < static_cast<uint32_t>(m)) {
-        o[r] = static_cast<int32_t>(idx);
-        if (r == static_cast<uint32_t>(k - 1)) s.rec[0] = key;
-        if (r == static_cast<uint32_t>(a)) s.rec[1] = key;
+      bar_finish();  // bcnt[b] is now the end of bucket b (= start of b + 1)
+      const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
+      for (int e = fid; e < n; e += kFinishThreads) {
+        const uint32_t key = s.hkey[e], idx = s.hidx[e];
+        const uint64_t cc = comp(key, idx);
+        if (cc > cmax) continue;
+        const uint32_t b = static_cast<uint32_t>(cc >> sh);
+        const uint32_t s0 = b ? s.bcnt[b - 1] : 0u, s1 = s.bcnt[b];
+        if (s0 >= static_cast<uint32_t>(m)) continue;
+        uint32_t r = s0;
+        for (uint32_t q = s0; q < s1; ++q) {
+          const uint32_t j = s.perm[q];
+          const uint32_t kj = s.hkey[j], ij = s.hidx[j];
+          r += kj > key || (kj == key && ij < idx);
+        }
+        if (r < static_cast<uint32_t>(m)) {
+          o[r] = static_cast<int32_t>(idx);
+          if (r == static_cast<uint32_t>(k - 1)) s.rec[0] = key;
+          if (r == static_cast<uint32_t>(a)) s.rec[1] = key;
+        }
       }
+      bar_finish();
     }
-    bar_finish();
   }
   if (fid == 0) {
     bool ok = false;
@@ -867,17 +918,21 @@ __device__ void finish_loop(Smem& s, int64_t num_rows, int k, int32_t* __restric
 // ---------------------------------------------------------- producer warp
 __device__ void produce_loop(Smem& s, const float* logits, int64_t row_stride, const int32_t* lengths,
                              int64_t num_rows) {
-  uint32_t g = 0;
+  int slot = 0;         // ring slot of the next stage
+  uint32_t phase = 0u;  // parity of the slot's current fill
   for (int64_t row = blockIdx.x; row < num_rows; row += gridDim.x) {
     const int64_t L = clamp_len(lengths, row, row_stride);
     const RowSpan sp = row_span(logits + row * row_stride, L);
-    for (int st = 0; st < sp.nst; ++st, ++g) {
-      const int slot = static_cast<int>(g % kStages);
-      mbar_wait_sleep(&s.empty[slot], ((g / kStages) & 1u) ^ 1u);
+    for (int st = 0; st < sp.nst; ++st) {
+      mbar_wait_sleep(&s.empty[slot], phase ^ 1u);
       const uint32_t bytes = st + 1 == sp.nst ? sp.last_bytes : kStageBytes;
       fence_proxy_async();
       mbar_arrive_expect_tx(&s.full[slot], bytes);
       bulk_g2s(&s.ring[slot][0], sp.src + static_cast<uint64_t>(st) * kStageBytes, bytes, &s.full[slot]);
+      if (++slot == kStages) {
+        slot = 0;
+        phase ^= 1u;
+      }
     }
   }
 }

@@ -220,6 +220,29 @@ def test_adversarial_orders(oracle_mod, dsa, pattern, rows):
     assert_parity(oracle_mod, dsa, x, L, 2048)
 
 
+@pytest.mark.parametrize("k", [2048, 512])
+def test_fp8_grid_many_rows(oracle_mod, dsa, k):
+    """Many rows of values on the fp8 e4m3 grid (heavy ties at every level):
+    the many-row path with its estimates carried between rows, and the
+    finisher's sorted fallback for buckets full of equal keys."""
+    rng = np.random.default_rng(77 + k)
+    rows, width = 296, 65536
+    x = workloads.round_to_e4m3(rng.standard_normal((rows, width))).astype(np.float32)
+    L = rng.integers(30000, width, size=rows, endpoint=True).astype(np.int32)
+    assert_parity(oracle_mod, dsa, x, L, k)
+
+
+def test_few_levels_many_rows(oracle_mod, dsa):
+    """Three distinct values over many rows: every bucket of the finisher's
+    first pass is one level, so the sorted fallback orders them by index."""
+    rng = np.random.default_rng(31)
+    x = (rng.integers(0, 3, (160, 50000)) * 1.0).astype(np.float32)
+    L = np.full(160, 50000, np.int32)
+    L[1::3] = 33333
+    assert_parity(oracle_mod, dsa, x, L, 2048)
+    assert_parity(oracle_mod, dsa, x, L, 100)
+
+
 def test_heavy_ties_cluster_exact_path(oracle_mod, dsa):
     """Few levels across a cluster-split row: the merge must split the tied
     threshold level across ranks in index order."""
