@@ -102,6 +102,23 @@ def profiled_traffic(config):
     return float(m_b.group(1))
 
 
+# ------------------------------------------------------------ rank logic
+def max_over_ranks(ms, dist=None, device="cpu"):
+    """The slowest rank's duration: every rank's timed region ends when all
+    have finished, so whole-job throughput divides by this."""
+    if dist is None:
+        return float(ms)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rows_per_s(world, rows_per_rank, steps, ms_max):
+    """Rows of all ranks per second (weak scaling: each rank its own batch)."""
+    return world * rows_per_rank * steps / (ms_max / 1e3)
+
+
 # ------------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and clock-event reasons via NVML (read-only) on a
@@ -263,10 +280,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dist if world > 1 else None, "cuda")
     status = dsa.device_status()
 
     # ---- end to end through the host-buffer C-ABI entry point
@@ -278,7 +292,7 @@ def run_ours(args):
     achieved = vb / per_launch_us / 1e3  # GB/s of valid logits
     result = {
         "metric": METRIC,
-        "value": round(world * wl.num_rows * args.steps / (ms_max / 1e3), 1),
+        "value": round(job_rows_per_s(world, wl.num_rows, args.steps, ms_max), 1),
         "unit": "rows/s",
         "n_gpus": world,
         "steps": args.steps,
