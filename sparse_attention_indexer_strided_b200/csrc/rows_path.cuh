@@ -361,7 +361,12 @@ __device__ __noinline__ uint32_t compact_exact(Smem& s, int n, int m, int tid) {
 // then keeps exactly those (a superset of the top m). Returns false, having
 // changed nothing, when that needs more than kRounds rounds or the bucket is
 // one tied key with too many entries: the exact pass must run.
-__device__ __noinline__ bool compact_fast(Smem& s, int n, int m, uint32_t& lo_out, uint32_t& kept, int tid) {
+struct FastCut {
+  uint32_t ok, lo, kept;
+};
+
+__device__ __noinline__ FastCut compact_fast(Smem& s, int n, int m, int tid) {
+  uint32_t kept = 0;
   const int w = tid >> 5, lane = tid & 31;
   bar_filter();  // every append is visible
   uint32_t lo, hi;
@@ -406,10 +411,9 @@ __device__ __noinline__ bool compact_fast(Smem& s, int n, int m, uint32_t& lo_ou
       break;
     }
   }
-  if (!ok) return false;
+  if (!ok) return FastCut{0u, 0u, 0u};
   keep_pass<false>(s, n, lo - 1u, 0u, tid);  // key >= lo (every real key is >= 1)
-  lo_out = lo;
-  return true;
+  return FastCut{1u, lo, kept};
 }
 
 struct Filter {
@@ -434,11 +438,11 @@ __device__ __forceinline__ void tighten(Filter& f, int m) {
 
 // Bounds the buffer again: the approximate pass, else the exact one.
 __device__ __forceinline__ void compact_any(Smem& s, Filter& f, int m, int tid) {
-  uint32_t lo = 0, kept = 0;
-  if (compact_fast(s, static_cast<int>(f.cnt), m, lo, kept, tid)) {
-    f.cnt = kept;
-    f.t = lo > kInfKey ? __int_as_float(0x7f800000) : from_key(lo);
-    f.last_key = lo;
+  const FastCut c = compact_fast(s, static_cast<int>(f.cnt), m, tid);
+  if (c.ok) {
+    f.cnt = c.kept;
+    f.t = c.lo > kInfKey ? __int_as_float(0x7f800000) : from_key(c.lo);
+    f.last_key = c.lo;
     f.strict = false;
     tighten(f, m);
   } else {
@@ -483,8 +487,10 @@ __device__ __forceinline__ void put_survivors(Smem& s, const float* src, uint32_
 // so the compaction applies; afterwards a half (<= kStageElems / 2) fits. Masks
 // taken before a compaction are supersets of the current ones, which is
 // harmless: the final ranking is exact.
+// (Rare paths take and return the filter state by value so that it never has
+// an address and stays in registers in the hot loop.)
 template <bool kRing>
-__device__ __noinline__ void take_stage_split(Smem& s, Filter& f, uint4 ra, uint4 rb, const float* src, uint32_t msk,
+__device__ __noinline__ Filter take_stage_split(Smem& s, Filter f, uint4 ra, uint4 rb, const float* src, uint32_t msk,
                                               uint32_t idx0, int m, int tid) {
   const int w = tid >> 5, lane = tid & 31;
   const uint32_t r[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
@@ -501,6 +507,7 @@ __device__ __noinline__ void take_stage_split(Smem& s, Filter& f, uint4 ra, uint
     f.cnt += tot;
     bar_filter();  // this half's entries are visible to a following compaction
   }
+  return f;
 }
 
 // Takes one stage after the filter barrier that completed its per-warp counts.
@@ -520,7 +527,7 @@ __device__ __forceinline__ void take_stage(Smem& s, Filter& f, const uint4* red,
     put_survivors<kRing>(s, src, msk, idx0, f.cnt + before, w, lane);
     f.cnt += tot;
   } else {
-    take_stage_split<kRing>(s, f, ra, rb, src, msk, idx0, m, tid);
+    f = take_stage_split<kRing>(s, f, ra, rb, src, msk, idx0, m, tid);
   }
 }
 
@@ -543,7 +550,7 @@ __device__ __forceinline__ uint32_t stage_mask(const float (&v)[kVals], float t,
 
 // The speculative threshold let fewer than m values through: stream the row
 // again from global memory with no threshold (one filter barrier per stage).
-__device__ __noinline__ void refilter_from_global(Smem& s, Filter& f, const RowSpan& sp, int64_t L, int m, int tid) {
+__device__ __noinline__ Filter refilter_from_global(Smem& s, Filter f, RowSpan sp, int64_t L, int m, int tid) {
   const int w = tid >> 5, lane = tid & 31;
   f.cnt = 0;
   f.t = __int_as_float(0xff800000);  // -inf: keep everything
@@ -573,6 +580,7 @@ __device__ __noinline__ void refilter_from_global(Smem& s, Filter& f, const RowS
     tighten(f, m);
   }
   bar_filter();
+  return f;
 }
 
 // A threshold for a row with no estimate, from a sample of kStageElems values
@@ -673,7 +681,7 @@ __device__ void filter_loop(Smem& s, const float* logits, int64_t row_stride, co
       }
     }
     bar_filter();  // every append is visible
-    if (spec && !f.compacted && f.cnt < static_cast<uint32_t>(m)) refilter_from_global(s, f, sp, L, m, tid);
+    if (spec && !f.compacted && f.cnt < static_cast<uint32_t>(m)) f = refilter_from_global(s, f, sp, L, m, tid);
     if (f.cnt > static_cast<uint32_t>(kHandCap)) compact_any(s, f, m, tid);
     if (tid == 0 && m == k && f.compacted) {
       s.own_key = f.last_key;
