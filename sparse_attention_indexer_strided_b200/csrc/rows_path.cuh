@@ -14,7 +14,7 @@
 //                                  later equal key has a larger index, so it
 //                                  loses its tie). At the end of the row the
 //                                  candidates are handed to the finishers.
-//   finisher (4 warps)           : ranks the handed-over candidates by (key
+//   finisher (6 warps)           : ranks the handed-over candidates by (key
 //                                  descending, index ascending) with a bucket
 //                                  pass over a composite key and writes the
 //                                  first m indices, -1 padding, while the
@@ -34,10 +34,10 @@ namespace rows {
 
 constexpr int kFilterWarps = 8;
 constexpr int kFilterThreads = kFilterWarps * 32;  // 256
-constexpr int kFinishWarps = 4;
-constexpr int kFinishThreads = kFinishWarps * 32;  // 128
+constexpr int kFinishWarps = 6;
+constexpr int kFinishThreads = kFinishWarps * 32;  // 192
 constexpr int kProducerWarp = kFilterWarps + kFinishWarps;
-constexpr int kThreads = (kProducerWarp + 1) * 32;  // 416
+constexpr int kThreads = (kProducerWarp + 1) * 32;  // 480
 constexpr int kGroups = 8;                              // float4 groups per lane and stage
 constexpr int kVals = 4 * kGroups;                      // 32 values per lane and stage
 constexpr int kWarpElems = 32 * kVals;                  // 1024 per warp and stage
@@ -47,7 +47,7 @@ constexpr int kStages = 3;                              // 96 KB ring
 constexpr int kFiltCap = 8192;                          // candidate buffer entries
 constexpr int kTrigger = kFiltCap / 2;                  // compact after a stage that leaves more
 constexpr int kHandCap = 4096;                          // handed-over candidates, at most
-constexpr int kBuckets = 4096;                          // finisher bucket counters (32 per thread)
+constexpr int kBuckets = 3840;                          // finisher bucket counters (20 per thread)
 constexpr int kPerThread = kFiltCap / kFilterThreads;   // 32 entries per filter thread
 constexpr int kScanPer = kBuckets / kFinishThreads;     // 32 counters per finisher thread
 constexpr uint32_t kInfKey = 0xFF800000u;               // key of +inf
@@ -73,6 +73,7 @@ struct __align__(128) Smem {
   uint32_t hidx[kHandCap];
   uint32_t bcnt[kBuckets];  // finisher bucket counters / ends
   uint16_t perm[kHandCap];  // finisher: candidates grouped by bucket
+  int32_t ostage[kMaxK];    // finisher: the row's output, written out coalesced
   uint32_t hist[256];       // filter radix histogram
   uint4 red[2][kFilterWarps / 4];  // per-warp survivor counts, by stage parity
   uint32_t fred[4][kFilterWarps];
@@ -888,12 +889,13 @@ __device__ void finish_one(Smem& s, int k, int32_t* __restrict__ out, int h, int
           r += kj > key || (kj == key && ij < idx);
         }
         if (r < static_cast<uint32_t>(m)) {
-          o[r] = static_cast<int32_t>(idx);
+          s.ostage[r] = static_cast<int32_t>(idx);
           if (r == static_cast<uint32_t>(k - 1)) s.rec[0] = key;
           if (r == static_cast<uint32_t>(a)) s.rec[1] = key;
         }
       }
       bar_finish();
+      for (int p = fid; p < m; p += kFinishThreads) o[p] = s.ostage[p];
     }
   }
   if (fid == 0) {
