@@ -48,7 +48,7 @@ constexpr int kFiltCap = 8192;                          // candidate buffer entr
 constexpr int kTrigger = kFiltCap / 2;                  // compact after a stage that leaves more
 constexpr int kHandCap = 4096;                          // handed-over candidates, at most
 constexpr int kBuckets = 3840;                          // finisher bucket counters (20 per thread)
-constexpr int kPerThread = kFiltCap / kFilterThreads;   // 32 entries per filter thread
+constexpr int kPerThread = (kFiltCap + kFilterThreads - 1) / kFilterThreads;  // entries per filter thread
 constexpr int kScanPer = kBuckets / kFinishThreads;     // 32 counters per finisher thread
 constexpr uint32_t kInfKey = 0xFF800000u;               // key of +inf
 constexpr int kRounds = 4;                              // radix rounds of 8 bits
@@ -61,6 +61,7 @@ constexpr int kSortPasses = 3;                          // finisher: bucket coun
 
 static_assert(kVals <= 32, "a lane's survivors of one stage form a 32-bit mask");
 static_assert(kFiltCap - kTrigger >= kStageElems / 2, "half a stage fits after a compaction");
+static_assert(kFilterWarps % 2 == 0 && kKeepLimit + kStageElems / 2 <= kFiltCap, "split halves fit after a compaction");
 static_assert(kHandCap >= kMaxK && kTrigger >= kMaxK, "buffers must hold k entries");
 static_assert(kBuckets == kScanPer * kFinishThreads && kBuckets <= 4096 && kScanPer % 4 == 0,
               "bucket counters split evenly over the finisher threads");
@@ -75,7 +76,7 @@ struct __align__(128) Smem {
   uint16_t perm[kHandCap];  // finisher: candidates grouped by bucket
   int32_t ostage[kMaxK];    // finisher: the row's output, written out coalesced
   uint32_t hist[256];       // filter radix histogram
-  uint4 red[2][kFilterWarps / 4];  // per-warp survivor counts, by stage parity
+  uint4 red[2][(kFilterWarps + 3) / 4];  // per-warp survivor counts, by stage parity
   uint32_t fred[4][kFilterWarps];
   uint32_t nred[5][kFinishWarps];
   uint32_t bc[8];
@@ -97,7 +98,7 @@ struct __align__(128) Smem {
 };
 static_assert(sizeof(Smem) <= 232448, "shared memory budget of one CTA per SM");
 
-__device__ __forceinline__ void bar_filter() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void bar_filter() { asm volatile("bar.sync 1, %0;" ::"n"(kFilterThreads) : "memory"); }
 __device__ __forceinline__ void bar_finish() { asm volatile("bar.sync 2, %0;" ::"n"(kFinishThreads) : "memory"); }
 
 // Warp sum by shuffles (the per-stage path avoids redux.sync, whose
@@ -211,7 +212,7 @@ __device__ uint32_t filter_kth(Smem& s, int n, uint32_t need, V v, P pred, int t
       break;
     }
     const int sh = window_shift(lo, hi);
-    s.hist[tid] = 0u;  // 256 filter threads, 256 bins
+    for (int i = tid; i < 256; i += kFilterThreads) s.hist[i] = 0u;
     if (tid == 0) {
       s.bc[0] = 0xFFFFFFFFu;
       s.bc[2] = 0u;
@@ -376,7 +377,7 @@ __device__ __noinline__ FastCut compact_fast(Smem& s, int n, int m, int tid) {
   bool ok = false;
   for (int round = 0; round < kRounds && lo != hi; ++round) {
     const int sh = window_shift(lo, hi);
-    s.hist[tid] = 0u;
+    for (int i = tid; i < 256; i += kFilterThreads) s.hist[i] = 0u;
     if (tid == 0) s.bc[0] = 0xFFFFFFFFu;
     bar_filter();
     uint32_t cur = 0xFFFFFFFFu, run = 0;
@@ -483,7 +484,7 @@ __device__ __forceinline__ void put_survivors(Smem& s, const float* src, uint32_
 
 // A stage whose survivors do not fit behind the buffer's contents (rare: no
 // usable threshold yet, or values rising along the row): the warps write in
-// two halves of four, compacting first whenever a half would not fit. A half
+// two halves, compacting first whenever a half would not fit. A half
 // with more than the free space implies more than kTrigger >= m entries held,
 // so the compaction applies; afterwards a half (<= kStageElems / 2) fits. Masks
 // taken before a compaction are supersets of the current ones, which is
@@ -491,20 +492,21 @@ __device__ __forceinline__ void put_survivors(Smem& s, const float* src, uint32_
 // (Rare paths take and return the filter state by value so that it never has
 // an address and stays in registers in the hot loop.)
 template <bool kRing>
-__device__ __noinline__ Filter take_stage_split(Smem& s, Filter f, uint4 ra, uint4 rb, const float* src, uint32_t msk,
+__device__ __noinline__ Filter take_stage_split(Smem& s, Filter f, const uint32_t* red, const float* src, uint32_t msk,
                                               uint32_t idx0, int m, int tid) {
+  constexpr int kHalf = kFilterWarps / 2;
   const int w = tid >> 5, lane = tid & 31;
-  const uint32_t r[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
   for (int half = 0; half < 2; ++half) {
     uint32_t tot = 0, before = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int ww = 4 * half + i;
-      tot += r[ww];
-      before += ww < w ? r[ww] : 0u;
+    for (int i = 0; i < kHalf; ++i) {
+      const int ww = kHalf * half + i;
+      const uint32_t c = red[ww];
+      tot += c;
+      before += ww < w ? c : 0u;
     }
     if (f.cnt + tot > static_cast<uint32_t>(kFiltCap)) compact_any(s, f, m, tid);
-    if ((w >> 2) == half) put_survivors<kRing>(s, src, msk, idx0, f.cnt + before, w, lane);
+    if (w / kHalf == half) put_survivors<kRing>(s, src, msk, idx0, f.cnt + before, w, lane);
     f.cnt += tot;
     bar_filter();  // this half's entries are visible to a following compaction
   }
@@ -516,8 +518,15 @@ template <bool kRing>
 __device__ __forceinline__ void take_stage(Smem& s, Filter& f, const uint4* red, const float* src, uint32_t msk,
                                            uint32_t idx0, int m, int tid) {
   const int w = tid >> 5, lane = tid & 31;
-  const uint4 ra = red[0], rb = red[1];
-  const uint32_t r[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+  uint32_t r[4 * ((kFilterWarps + 3) / 4)];
+#pragma unroll
+  for (int i = 0; i < (kFilterWarps + 3) / 4; ++i) {
+    const uint4 q = red[i];
+    r[4 * i + 0] = q.x;
+    r[4 * i + 1] = q.y;
+    r[4 * i + 2] = q.z;
+    r[4 * i + 3] = q.w;
+  }
   uint32_t before = 0, tot = 0;
 #pragma unroll
   for (int i = 0; i < kFilterWarps; ++i) {
@@ -528,7 +537,7 @@ __device__ __forceinline__ void take_stage(Smem& s, Filter& f, const uint4* red,
     put_survivors<kRing>(s, src, msk, idx0, f.cnt + before, w, lane);
     f.cnt += tot;
   } else {
-    f = take_stage_split<kRing>(s, f, ra, rb, src, msk, idx0, m, tid);
+    f = take_stage_split<kRing>(s, f, reinterpret_cast<const uint32_t*>(red), src, msk, idx0, m, tid);
   }
 }
 
