@@ -89,8 +89,8 @@ struct __align__(128) Smem {
   int64_t est_len[2];
   float est[2];
   int32_t est_ok[2];
-  // the filter warps' own estimate: the last compaction of an earlier row kept
-  // at least k keys >= own_key (own_len 0: none yet)
+  // the filter warps' own estimate: an earlier row of length own_len held at
+  // least k candidates with key >= own_key (own_len 0: none yet)
   uint32_t own_key;
   int32_t own_len;
   unsigned long long full[kStages], empty[kStages];
@@ -424,7 +424,8 @@ struct Filter {
   int par;            // stage parity of s.red on the synchronous path
   bool compacted;     // the row was compacted at least once
   bool strict;        // t already excludes values equal to the held m-th key
-  uint32_t last_key;  // the last compaction kept every key >= last_key, at least m of them
+  bool bounded;       // last_key is set
+  uint32_t last_key;  // at least m candidates with key >= last_key are held
 };
 
 // Holding at least m candidates, every one at or above the threshold t: a
@@ -433,7 +434,9 @@ struct Filter {
 // filling the buffer).
 __device__ __forceinline__ void tighten(Filter& f, int m) {
   if (!f.strict && m > 0 && f.cnt >= static_cast<uint32_t>(m)) {
-    f.t = above(to_key(f.t));
+    f.last_key = to_key(f.t);
+    f.bounded = true;
+    f.t = above(f.last_key);
     f.strict = true;
   }
 }
@@ -445,6 +448,7 @@ __device__ __forceinline__ void compact_any(Smem& s, Filter& f, int m, int tid) 
     f.cnt = c.kept;
     f.t = c.lo > kInfKey ? __int_as_float(0x7f800000) : from_key(c.lo);
     f.last_key = c.lo;
+    f.bounded = true;
     f.strict = false;
     tighten(f, m);
   } else {
@@ -452,6 +456,7 @@ __device__ __forceinline__ void compact_any(Smem& s, Filter& f, int m, int tid) 
     f.cnt = static_cast<uint32_t>(m);
     f.t = above(T);
     f.last_key = T;
+    f.bounded = true;
     f.strict = true;
   }
   f.compacted = true;
@@ -566,6 +571,7 @@ __device__ __noinline__ Filter refilter_from_global(Smem& s, Filter f, RowSpan s
   f.t = __int_as_float(0xff800000);  // -inf: keep everything
   f.compacted = false;
   f.strict = false;
+  f.bounded = false;
   for (int st = 0; st < sp.nst; ++st) {
     const float* src = reinterpret_cast<const float*>(sp.src + static_cast<uint64_t>(st) * kStageBytes);
     const uint32_t avail = st + 1 == sp.nst ? sp.last_bytes : kStageBytes;
@@ -671,6 +677,7 @@ __device__ void filter_loop(Smem& s, const float* logits, int64_t row_stride, co
     f.cnt = 0;
     f.compacted = false;
     f.strict = false;
+    f.bounded = false;
     int32_t sj0 = static_cast<int32_t>(sp.j0);  // row index of the stage's first float (< L <= INT32_MAX)
     for (int st = 0; st < sp.nst; ++st, sj0 += kStageElems) {
       mbar_wait(&s.full[slot], phase);
@@ -693,7 +700,7 @@ __device__ void filter_loop(Smem& s, const float* logits, int64_t row_stride, co
     bar_filter();  // every append is visible
     if (spec && !f.compacted && f.cnt < static_cast<uint32_t>(m)) f = refilter_from_global(s, f, sp, L, m, tid);
     if (f.cnt > static_cast<uint32_t>(kHandCap)) compact_any(s, f, m, tid);
-    if (tid == 0 && m == k && f.compacted) {
+    if (tid == 0 && m == k && f.bounded) {
       s.own_key = f.last_key;
       s.own_len = L;
     }
