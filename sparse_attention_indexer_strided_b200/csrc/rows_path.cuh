@@ -464,26 +464,38 @@ __device__ __forceinline__ void compact_any(Smem& s, Filter& f, int m, int tid) 
 
 // Writes this warp's survivors (bit j of msk: value j of the lane; values
 // re-read from src, the stage in the ring or in global memory) at positions
-// pos.., one survivor per lane and round.
+// pos.., up to two survivors per lane and round.
 template <bool kRing>
 __device__ __forceinline__ void put_survivors(Smem& s, const float* src, uint32_t msk, uint32_t idx0, uint32_t pos,
                                               int w, int lane) {
   const uint32_t lt = lanemask_lt();
   uint32_t rest = msk;
-  for (;;) {
-    const bool act = rest != 0u;
-    const uint32_t bal = __ballot_sync(kFull, act);
-    if (bal == 0u) break;
-    if (act) {
-      const int j = __ffs(rest) - 1;
-      rest &= rest - 1u;
-      const int off = val_offset(w, lane, j);
-      const uint32_t p = pos + __popc(bal & lt);
-      const float x = kRing ? src[off] : __ldg(src + off);
-      s.fkey[p] = to_key(x);
-      s.fidx[p] = idx0 + static_cast<uint32_t>(off);
+  for (;;) {  // two survivors per lane and iteration: their loads overlap
+    const bool a1 = rest != 0u;
+    const uint32_t b1 = __ballot_sync(kFull, a1);
+    if (b1 == 0u) break;
+    const int j1 = __ffs(rest) - 1;
+    rest &= rest - 1u;
+    const bool a2 = rest != 0u;
+    const uint32_t b2 = __ballot_sync(kFull, a2);
+    const int j2 = __ffs(rest) - 1;
+    rest &= rest - 1u;
+    const uint32_t n1 = __popc(b1);
+    const int o1 = val_offset(w, lane, j1 & 31), o2 = val_offset(w, lane, j2 & 31);
+    float x1 = 0.f, x2 = 0.f;
+    if (a1) x1 = kRing ? src[o1] : __ldg(src + o1);
+    if (a2) x2 = kRing ? src[o2] : __ldg(src + o2);
+    if (a1) {
+      const uint32_t p = pos + __popc(b1 & lt);
+      s.fkey[p] = to_key(x1);
+      s.fidx[p] = idx0 + static_cast<uint32_t>(o1);
     }
-    pos += __popc(bal);
+    if (a2) {
+      const uint32_t p = pos + n1 + __popc(b2 & lt);
+      s.fkey[p] = to_key(x2);
+      s.fidx[p] = idx0 + static_cast<uint32_t>(o2);
+    }
+    pos += n1 + __popc(b2);
   }
 }
 
