@@ -941,6 +941,88 @@ __device__ __noinline__ uint32_t stream_global(Smem& s, const Span& sp, int64_t 
   return st.count;
 }
 
+// need-th largest key among candidates [0, n) (consumer threads; 1 <= need
+// <= n): the radix rounds of select_topk without the compaction.
+__device__ __noinline__ uint32_t kth_key(Smem& s, int n, uint32_t need, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  const MinMax r = block_minmax(s, 0, n, tid);
+  uint32_t lo = r.mn, hi = r.mx;
+  for (int round = 0; lo != hi; ++round) {
+    if (round == kMaxRadixRounds) {
+      if (tid == 0) atomicOr(&g_status, kStatusSelectBroken);
+      break;
+    }
+    const int sh = window_shift(lo, hi);
+    if (tid < 256) s.hist[tid] = 0u;
+    if (tid == 0) {
+      s.bc[0] = 0xFFFFFFFFu;
+      s.bc[2] = 0u;
+    }
+    __syncthreads();
+    histogram(s, s.hist, 0, n, lo, hi, sh, tid);
+    __syncthreads();
+    if (w == 0) find_bucket_warp0(s.hist, need, s.bc, lane);
+    __syncthreads();
+    const uint32_t b = s.bc[0], above_b = s.bc[1];
+    if (b == 0xFFFFFFFFu) {
+      if (tid == 0) atomicOr(&g_status, kStatusSelectBroken);
+      break;
+    }
+    const uint32_t in_bucket = s.hist[b];
+    need -= above_b;
+    narrow(lo, hi, sh, b);
+    if (in_bucket <= 32u && lo != hi) {
+      for (int e = tid; e < n; e += kConsumerThreads) {
+        const uint32_t key = s.ckey[e];
+        if (key >= lo && key <= hi) {
+          const uint32_t slot = atomicAdd(&s.bc[2], 1u);
+          if (slot < 32u) s.small[slot] = key;
+        }
+      }
+      __syncthreads();
+      if (w == 0) {
+        const uint32_t t = small_kth(lane < static_cast<int>(in_bucket) ? s.small[lane] : 0u, need);
+        if (lane == 0) s.bc[3] = t;
+      }
+      __syncthreads();
+      lo = hi = s.bc[3];
+    }
+    __syncthreads();
+  }
+  return lo;
+}
+
+// A starting threshold for a cluster rank's chunk [c0, c1) of a row: the
+// chunk is sampled as kStageElems values in 32 evenly spaced runs of 128
+// (aligned 16-byte blocks inside the chunk), and the threshold is the value
+// with 1.5 times the chunk's share of m_r sampled values above it, plus 16.
+// Returns -inf when the sample gives none.
+__device__ __noinline__ float chunk_threshold(Smem& s, const float* row, int64_t c0, int64_t c1, uint32_t m_r,
+                                              int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(row + c0);
+  const uintptr_t as = a & ~static_cast<uintptr_t>(15);
+  const int64_t j0 = c0 - static_cast<int64_t>((a - as) >> 2);  // row index of the aligned base
+  const int64_t span = c1 - j0;                                   // floats from there to the chunk end
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int64_t run = w * 4 + q;  // 0..31
+    const int64_t b = ((span - 128) * run / 31) & ~static_cast<int64_t>(3);
+    const float4 x = __ldg(reinterpret_cast<const float4*>(as) + (b >> 2) + lane);
+    const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t j = j0 + b + 4 * lane + i;
+      s.ckey[w * 512 + q * 128 + lane * 4 + i] = (j >= c0 && j < c1) ? to_key(xv[i]) : 0u;  // 0: below every key
+    }
+  }
+  __syncthreads();
+  const double share = static_cast<double>(kStageElems) * m_r / static_cast<double>(c1 - c0);
+  const uint32_t need = min(static_cast<uint32_t>(kStageElems - 8), static_cast<uint32_t>(1.5 * share) + 16u);
+  const uint32_t T = kth_key(s, kStageElems, need, tid);
+  return (T == 0u || T >= 0xFF800000u) ? __int_as_float(0xff800000) : from_key(T);
+}
+
 __device__ __forceinline__ void init_pipeline(Smem& s) {
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) mbar_init(&s.full[i], 1);
@@ -951,6 +1033,12 @@ __device__ __forceinline__ void init_pipeline(Smem& s) {
 
 // --------------------------------------------------------------- kernels
 // Few long rows: a cluster of CTAs per row (grid = num_rows * cluster size).
+// kSample: ranks whose chunk holds at least kSampleChunk values start from a
+// sampled threshold; the host picks the instantiation from row_stride and the
+// cluster size (which bound every chunk), so short chunks run the plain one.
+constexpr int64_t kSampleChunk = 8 * kStageElems;
+
+template <bool kSample>
 __global__ void __launch_bounds__(kThreads, kBlocksPerSM)
     topk_cluster_kernel(const float* __restrict__ logits, int64_t row_stride, const int32_t* __restrict__ lengths,
                         int64_t num_rows, int k, int32_t* __restrict__ out) {
@@ -984,11 +1072,26 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM)
     producer_set_item(prod, is);
     for (int i = 0; i < kStages; ++i) producer_issue(s, prod, is);
   }
+  // a sampled starting threshold for long chunks (the ring is already filling)
+  const uint32_t m_r = static_cast<uint32_t>(min64(k, c1 - c0));
+  int mode0 = kAcceptAll;
+  float thr0 = 0.f;
+  if (kSample && c1 - c0 >= kSampleChunk && m_r > 0) {
+    const float t = chunk_threshold(s, row_ptr, c0, c1, m_r, tid);
+    if (t > __int_as_float(0xff800000)) {
+      mode0 = kAtLeast;
+      thr0 = t;
+    }
+  }
   uint32_t g = 0;
   int par = 0;
   bool compacted = false;
-  uint32_t n_r = stream_ring(s, sp, c0, c1, k, g, par, kAcceptAll, 0.f, compacted, tid, tid == 0 ? &prod : nullptr,
+  uint32_t n_r = stream_ring(s, sp, c0, c1, k, g, par, mode0, thr0, compacted, tid, tid == 0 ? &prod : nullptr,
                              &is);
+  if (kSample && mode0 == kAtLeast && !compacted && n_r < m_r) {
+    // the sample's threshold let fewer than this rank's top-m_r through: redo exactly
+    n_r = stream_global(s, sp, c0, c1, k, par, tid);
+  }
   if (n_r > static_cast<uint32_t>(k)) {
     select_topk(s, 0, static_cast<int>(n_r), k, tid);
     n_r = static_cast<uint32_t>(k);
@@ -1154,7 +1257,9 @@ static int device_setup(int dev, DeviceInfo* out) {
     const int smem = static_cast<int>(sizeof(Smem));
     if (cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sizeof(rows::Smem))) != cudaSuccess ||
-        cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaFuncSetAttribute(topk_cluster_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(topk_cluster_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
             cudaSuccess) {
       cudaGetLastError();
       return DSA_ERR_CONFIG;
@@ -1162,8 +1267,10 @@ static int device_setup(int dev, DeviceInfo* out) {
     d.max_cluster = 0;
     for (int cs : {16, 8}) {
       if (cs > 8 &&
-          cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-              cudaSuccess) {
+          (cudaFuncSetAttribute(topk_cluster_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+               cudaSuccess ||
+           cudaFuncSetAttribute(topk_cluster_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+               cudaSuccess)) {
         cudaGetLastError();
         continue;
       }
@@ -1179,7 +1286,8 @@ static int device_setup(int dev, DeviceInfo* out) {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int nclusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&nclusters, topk_cluster_kernel, &cfg) == cudaSuccess && nclusters > 0) {
+      if (cudaOccupancyMaxActiveClusters(&nclusters, topk_cluster_kernel<false>, &cfg) == cudaSuccess &&
+          nclusters > 0) {
         d.max_cluster = cs;
         break;
       }
@@ -1257,8 +1365,14 @@ static int launch(const DeviceInfo& d, const float* logits, int64_t row_stride, 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, logits, row_stride, lengths, num_rows, static_cast<int>(k),
-                           out);
+    // the longest possible chunk decides whether any rank samples
+    const int64_t max_chunk = (row_stride + cs - 1) / cs;
+    if (max_chunk >= kSampleChunk)
+      e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<true>, logits, row_stride, lengths, num_rows,
+                             static_cast<int>(k), out);
+    else
+      e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<false>, logits, row_stride, lengths, num_rows,
+                             static_cast<int>(k), out);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
