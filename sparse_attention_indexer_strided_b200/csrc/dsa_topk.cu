@@ -5,32 +5,26 @@
 // largest of the first L_r values, as row-local indices ordered by value
 // descending and index ascending, padded with -1 past min(k, L_r).
 //
-// Design (one HBM pass, no global scratch):
-//   * One producer warp streams a row (or a chunk of it) into a ring of
-//     shared-memory stages with cp.async.bulk (TMA bulk copies, no
-//     multicast) completing on mbarriers.
-//   * Consumer warps turn each fp32 into an order-preserving uint32
-//     key only when it can still matter: a running threshold T (the exact
-//     k-th largest key among the entries seen so far) filters the stream, and
-//     survivors are appended to a shared-memory candidate buffer in index
-//     order. Because tiles arrive in index order, a later entry equal to T
-//     always loses its tie, so the filter is "key > T".
-//   * When the buffer would overflow, a radix select (adaptive 8-bit windows
-//     over the key range actually present) finds the exact k-th key, and a
-//     stable compaction keeps the k winners, ties by lowest index. This is
+// Design (one HBM pass, no global scratch), two kernels:
+//   * Many rows (rows_path.cuh, topk_rows_kernel): one persistent CTA per SM
+//     with a TMA producer warp, filter warps that stream each row against a
+//     running threshold into a shared candidate buffer, and finisher warps
+//     that rank the previous row's candidates while the next row streams.
+//   * Few long rows (this file, topk_cluster_kernel): a thread-block cluster
+//     splits a row into contiguous chunks. Each rank streams its chunk
+//     through a TMA ring (one producer thread issues cp.async.bulk copies, no
+//     multicast), keeps candidates above a running threshold in index order,
+//     and compacts with a radix select (adaptive 8-bit windows over the key
+//     range present) plus a stable keep that gives ties to the lowest index:
 //     the pages' histogram / run_cumsum / threshold / gt-eq split, made exact
-//     and deterministic.
-//   * At the end a stable LSD radix sort orders the <= k winners and the
-//     output row is written with -1 padding.
-//   * Many rows: one CTA per row, persistent over rows; the producer runs
-//     ahead into the next row while consumers finish the current one.
-//   * Few long rows: a thread-block cluster splits a row into contiguous
-//     chunks. Ranks merge through distributed shared memory: a cluster-wide
-//     histogram over the candidates narrows the threshold, ranks publish
-//     counts, and each rank writes its survivors into the leader's shared
-//     memory at rank-ordered offsets (so index order, hence the tie rule, is
-//     preserved). Cluster barriers separate the phases; every CTA reaches
-//     every barrier.
+//     and deterministic. Long chunks start from a sampled threshold. Ranks
+//     then merge through distributed shared memory: a cluster-wide histogram
+//     over the candidates narrows the threshold, ranks publish counts, and
+//     each rank writes its survivors into the leader's shared memory at
+//     rank-ordered offsets (so index order, hence the tie rule, is kept). The
+//     leader sorts the winners (stable LSD radix) and writes the row with -1
+//     padding. Cluster barriers separate the phases; every CTA reaches every
+//     barrier.
 //
 // Coding rules taken from the SGLang PR #34167 discussion: a distributed
 // shared-memory address is only ever a 32-bit shared::cluster address used

@@ -1,35 +1,40 @@
 // Many-row path: one persistent CTA per SM, three warp roles.
 //
 //   producer (1 warp, one lane)  : cp.async.bulk copies of the CTA's rows, in
-//                                  16 KB stages, into a 6-stage shared ring
+//                                  32 KB stages, into a 3-stage shared ring
 //                                  (full / empty mbarriers).
-//   filter   (8 warps)           : every stage, each lane compares its 16
+//   filter   (8 warps)           : every stage, each lane compares its 32
 //                                  values with the row's running threshold t
-//                                  (keep x unless x < t; NaN always kept) and
-//                                  appends the survivors' (key, index) pairs
-//                                  to a candidate buffer. When the buffer
-//                                  passes half full, an exact radix select
-//                                  keeps the row's top-m of what was seen and
-//                                  t becomes "strictly above the m-th key" (a
-//                                  later equal key has a larger index, so it
-//                                  loses its tie). At the end of the row the
-//                                  candidates are handed to the finishers.
+//                                  (keep x unless x < t; NaN always kept); the
+//                                  warps meet at one barrier per stage to place
+//                                  the survivors' (key, index) pairs in a
+//                                  shared candidate buffer. Once m candidates
+//                                  at or above t are held, t becomes strict (a
+//                                  later equal value has a larger index, so it
+//                                  loses its tie). When the buffer passes half
+//                                  full it is compacted: an approximate radix
+//                                  cut when one suffices, else an exact select
+//                                  with the tie cut by index. At the end of the
+//                                  row the candidates are handed over.
 //   finisher (6 warps)           : ranks the handed-over candidates by (key
-//                                  descending, index ascending) with a bucket
-//                                  pass over a composite key and writes the
-//                                  first m indices, -1 padding, while the
-//                                  filter warps already stream the next row.
+//                                  descending, index ascending) with bucket
+//                                  passes over a composite key (a bitonic sort
+//                                  when a bucket stays crowded with equal
+//                                  keys), then writes the first m indices and
+//                                  -1 padding while the filter warps already
+//                                  stream the next row.
 //
-// A row starts with a speculative threshold taken from the row the finisher
-// completed two rows earlier (the value that is as far below that row's k-th
-// largest as its 3k/4-th largest is above it). If fewer than m values pass it,
-// the filter warps re-read the row from global memory with no threshold; the
-// result is exact either way, only the time changes.
+// A row starts with a speculative threshold: from the row the finisher
+// completed two rows earlier (half the gap between that row's 3k/4-th and
+// k-th largest below its k-th), else from the bound the filter held on its
+// previous row, else from a sample of the row itself. If fewer than m values
+// pass it, the filter warps re-read the row from global memory with no
+// threshold; the result is exact either way, only the time changes.
 //
-// The select follows the pages' histogram / cumulative-sum / threshold / gt-eq
-// split (SGLang PR #34167 code excerpt, the radix top-k kernel), made exact:
-// ties at the threshold go to the lowest indices (a second radix select over
-// the indices of the tied keys) instead of a capped tie list.
+// The selection follows the pages' histogram / cumulative-sum / threshold /
+// gt-eq split (SGLang PR #34167 code excerpt, the radix top-k kernel), made
+// exact: ties at the threshold go to the lowest indices (a second radix select
+// over the indices of the tied keys) instead of a capped tie list.
 namespace rows {
 
 constexpr int kFilterWarps = 8;
