@@ -77,14 +77,26 @@ def load_peaks():
     return 6650.0, "fallback (6.65 TB/s, earlier measurement on this pool)"
 
 
+def _code_only(text):
+    """Source text without comments and blank lines (the digest follows code)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = []
+    for line in text.splitlines():
+        line = re.sub(r"//.*$", "", line).rstrip()
+        if line.strip():
+            lines.append(line)
+    return "\n".join(lines)
+
+
 def source_sha():
-    """Digest of every kernel source file (a traffic figure is only valid for it)."""
+    """Digest of the code of every kernel source file (a traffic figure is only
+    valid for it); comment-only edits keep it."""
     csrc = os.path.join(ROOT, "sparse_attention_indexer_strided_b200", "csrc")
     h = hashlib.sha256()
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh", ".h")):
             h.update(name.encode())
-            h.update(open(os.path.join(csrc, name), "rb").read())
+            h.update(_code_only(open(os.path.join(csrc, name), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 
