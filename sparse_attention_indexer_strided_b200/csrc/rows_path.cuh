@@ -68,6 +68,7 @@ static_assert(kVals <= 32, "a lane's survivors of one stage form a 32-bit mask")
 static_assert(kFiltCap - kTrigger >= kStageElems / 2, "half a stage fits after a compaction");
 static_assert(kFilterWarps % 2 == 0 && kKeepLimit + kStageElems / 2 <= kFiltCap, "split halves fit after a compaction");
 static_assert(kHandCap >= kMaxK && kTrigger >= kMaxK, "buffers must hold k entries");
+static_assert(kBuckets >= 2048, "bucket_shift narrows a 12-bit slice by at most one more bit");
 static_assert(kBuckets == kScanPer * kFinishThreads && kBuckets <= 4096 && kScanPer % 4 == 0,
               "bucket counters split evenly over the finisher threads");
 
