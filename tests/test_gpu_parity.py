@@ -243,6 +243,45 @@ def test_few_levels_many_rows(oracle_mod, dsa):
     assert_parity(oracle_mod, dsa, x, L, 100)
 
 
+def _sample_runs(span, runs):
+    """Start offsets of the evenly spaced 128-value runs a first threshold is
+    sampled from (16-byte aligned rows and chunks)."""
+    return [((span - 128) * r // (runs - 1)) & ~3 for r in range(runs)]
+
+
+def test_sampled_threshold_fallback_many_rows(oracle_mod, dsa):
+    """Large values exactly where a row's first threshold is sampled, small
+    values elsewhere: the sampled threshold lets far fewer than k values
+    through, so the row must be re-read with no threshold, and the result must
+    still be exact."""
+    rng = np.random.default_rng(5)
+    rows, L, stride = 148, 120000, 131072  # one row per CTA: every row is a first row
+    x = (rng.standard_normal((rows, stride)) * 0.01).astype(np.float32)
+    for b in _sample_runs(L, 64):
+        x[:, b:b + 128] = 100.0 + rng.random((rows, 128), dtype=np.float32)
+    Ls = np.full(rows, L, np.int32)
+    assert_parity(oracle_mod, dsa, x, Ls, 2048)
+    assert dsa.device_status() == 0
+
+
+def test_sampled_threshold_fallback_cluster(oracle_mod, dsa):
+    """The same trap for the cluster path: every rank's sample lands on large
+    values, so every rank must re-read its chunk."""
+    rng = np.random.default_rng(6)
+    rows, L, stride, ranks = 4, 900000, 900096, 16
+    if dsa.plan(rows, stride, 1024)[0] != ranks:
+        pytest.skip("this GPU does not run 16-CTA clusters")
+    chunk = (-(-L // ranks) + 3) & ~3
+    x = (rng.standard_normal((rows, stride)) * 0.01).astype(np.float32)
+    for r in range(ranks):
+        c0, c1 = min(L, r * chunk), min(L, r * chunk + chunk)
+        for b in _sample_runs(c1 - c0, 32):
+            x[:, c0 + b:c0 + b + 128] = 100.0 + rng.random((rows, 128), dtype=np.float32)
+    Ls = np.full(rows, L, np.int32)
+    assert_parity(oracle_mod, dsa, x, Ls, 1024)
+    assert dsa.device_status() == 0
+
+
 def test_heavy_ties_cluster_exact_path(oracle_mod, dsa):
     """Few levels across a cluster-split row: the merge must split the tied
     threshold level across ranks in index order."""
