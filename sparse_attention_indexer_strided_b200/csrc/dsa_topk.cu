@@ -585,13 +585,37 @@ __device__ __noinline__ uint32_t select_topk(Smem& s, int base, int n, int k, in
 __device__ __noinline__ int sort_desc(Smem& s, int src, int alt, int m, int tid) {
   const int w = tid >> 5, lane = tid & 31;
   if (m <= 1) return src;
-  const MinMax mm = block_minmax(s, src, m, tid);
-  if (mm.mn == mm.mx) return src;
-  const int passes = (31 - __clz(mm.mn ^ mm.mx)) / 8 + 1;
+  // bits that differ between some two keys: a byte with none is equal in every
+  // key, and its stable pass would be the identity (the low bytes of values on
+  // a coarse grid, such as fp8, are)
+  uint32_t any1 = 0u, all1 = 0xFFFFFFFFu;
+  for (int e = tid; e < m; e += kConsumerThreads) {
+    const uint32_t key = s.ckey[src + e];
+    any1 |= key;
+    all1 &= key;
+  }
+  any1 = __reduce_or_sync(kFull, any1);
+  all1 = __reduce_and_sync(kFull, all1);
+  if (lane == 0) {
+    s.red[2][w] = any1;
+    s.red[3][w] = all1;
+  }
+  __syncthreads();
+  any1 = 0u;
+  all1 = 0xFFFFFFFFu;
+#pragma unroll
+  for (int ww = 0; ww < kNumConsumerWarps; ++ww) {
+    any1 |= s.red[2][ww];
+    all1 &= s.red[3][ww];
+  }
+  const uint32_t varying = any1 & ~all1;
+  __syncthreads();  // red[2..3] may be rewritten by a later call
+  if (varying == 0u) return src;
   uint32_t* wcnt = s.ckey + kSortCountOff;  // [warp][256]
   const uint32_t lt = lanemask_lt();
-  for (int pass = 0; pass < passes; ++pass) {
+  for (int pass = 0; pass < 4; ++pass) {
     const int sh = pass * 8;
+    if (((varying >> sh) & 255u) == 0u) continue;  // the same byte in every key
 #pragma unroll
     for (int i = 0; i < 8; ++i) wcnt[w * 256 + i * 32 + lane] = 0u;
     __syncwarp();
