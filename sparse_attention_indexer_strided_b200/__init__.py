@@ -23,7 +23,7 @@ MAX_K = 2048
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        "libdsa_topk.so is not built; run `python -m sparse_attention_indexer_strided_b200.build` "
+        "libdsa_topk.so is not built; run `python sparse_attention_indexer_strided_b200/build.py` "
         "(nvcc, sm_100a). There is no CPU fallback.")
 
 _lib = ctypes.CDLL(LIB_PATH)

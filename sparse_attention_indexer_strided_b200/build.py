@@ -1,6 +1,9 @@
 """Ahead-of-time build of the CUDA library (sm_100a) into this package folder.
 
-    python -m sparse_attention_indexer_strided_b200.build [--force]
+    python sparse_attention_indexer_strided_b200/build.py [--force] [-v]
+
+Run it as a script (or load it by file path): the package itself cannot be
+imported before the library exists.
 
 nvcc cross-compiles without a GPU. The shared object keeps every symbol hidden
 except the C ABI declared in include/dsa_topk.h.

@@ -22,9 +22,9 @@ def declared_functions():
 
 @pytest.fixture(scope="module")
 def pkg():
-    from sparse_attention_indexer_strided_b200 import build
+    import __graft_entry__
 
-    build.build()
+    __graft_entry__.build()
     import sparse_attention_indexer_strided_b200 as m
     return m
 
