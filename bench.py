@@ -9,9 +9,11 @@ One step = one ``dsa_topk`` call over the whole batch of the chosen workload
 the inputs already resident in HBM. The prefill input (2.15 GB) is larger than
 the 126 MB L2, so consecutive steps read HBM; no flush is needed.
 
-Prints one JSON line (rank 0). ``value`` is rows/s over all ranks (weak
-scaling: every rank processes its own batch; there is no collective on the data
-path, only the max-over-ranks reduction of the timings). The line also carries
+Prints one JSON line (rank 0). ``value`` is rows/s over all ranks. By default
+every rank processes its own copy of the batch (weak scaling). With
+``--shard rows`` one batch is split into contiguous row blocks, one per rank,
+each rank holding only its own rows (strong scaling). Neither mode has a
+collective on the data path, only the max-over-ranks reduction of the timings. The line also carries
 the HBM roofline of the kernel, the oracle's CPU throughput on a bounded sample
 (N=1), the host-buffer end-to-end throughput, SM clocks sampled during the
 timed region, and per-workload timings of all five workloads (N=1).
@@ -60,6 +62,8 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=5, help="0 skips the host-buffer run")
     p.add_argument("--rows", type=int, default=0, help="use only the first N rows (profiling runs)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--shard", choices=["none", "rows"], default="none",
+                   help="rows: split one batch into contiguous row blocks across ranks (strong scaling)")
     return p.parse_args()
 
 
@@ -129,6 +133,11 @@ def max_over_ranks(ms, dist=None, device="cpu"):
 def job_rows_per_s(world, rows_per_rank, steps, ms_max):
     """Rows of all ranks per second (weak scaling: each rank its own batch)."""
     return world * rows_per_rank * steps / (ms_max / 1e3)
+
+
+def sharded_rows_per_s(batch_rows, steps, ms_max):
+    """Rows of one batch split across ranks, per second of the slowest rank."""
+    return batch_rows * steps / (ms_max / 1e3)
 
 
 # ------------------------------------------------------------------- clocks
@@ -218,32 +227,52 @@ def time_graph(dsa, torch, calls, reps=5):
     return statistics.median(out)
 
 
+def _time_workload(dsa, torch, peak, wl, dtype=None, unsorted=False, table=False):
+    """CUDA-graph timing of one workload (rotating input copies whose total
+    exceeds 4x L2, so each call reads HBM), plus an L2-warm number."""
+    elem = 4 if dtype is None else 2
+    vb = workloads.valid_bytes(wl.lengths) * elem // 4
+    base = torch.from_numpy(wl.logits).cuda()
+    if dtype is not None:
+        base = base.to(dtype)
+    tensor_bytes = base.numel() * base.element_size()
+    R = max(1, min(64, -(-4 * L2_BYTES // tensor_bytes)))
+    copies = [base] + [base.clone() for _ in range(R - 1)]
+    lengths = torch.from_numpy(wl.lengths).cuda()
+    out = torch.empty((wl.num_rows, wl.k), dtype=torch.int32, device="cuda")
+    tab = None
+    if table:  # a per-row lookup table (row-local index -> int32 value), made on the device
+        tab = torch.randint(0, 1 << 30, (wl.num_rows, wl.row_stride), dtype=torch.int32, device="cuda")
+    kw = {"unsorted": unsorted, "index_table": tab}
+    n_calls = max(R, min(256, max(8, int(2e9 // max(vb, 1)))))
+    cold = [(lambda c=copies[i % R]: dsa.dsa_topk(c, lengths, wl.k, out=out, **kw)) for i in range(n_calls)]
+    us_cold = time_graph(dsa, torch, cold)
+    warm = [(lambda: dsa.dsa_topk(base, lengths, wl.k, out=out, **kw)) for _ in range(min(n_calls, 64))]
+    us_warm = time_graph(dsa, torch, warm)
+    cs, grid = dsa.plan(wl.num_rows, wl.row_stride, wl.k)
+    gbs = vb / us_cold / 1e3
+    res = {
+        "us_per_call": round(us_cold, 3), "rows_per_s": round(wl.num_rows / us_cold * 1e6, 1),
+        "valid_gbs": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
+        "us_per_call_warm_l2": round(us_warm, 3), "valid_bytes": vb,
+        "rotating_copies": R, "cluster_size": cs, "grid": grid,
+    }
+    del copies, base, out, tab
+    torch.cuda.empty_cache()
+    return res
+
+
 def per_config_table(dsa, torch, peak):
+    """All five workloads, then the prefill workload with each call option:
+    bf16 logits (2 bytes per valid logit), the unsorted (set) output, and an
+    index table applied to every output."""
     rows = {}
     for name in workloads.CONFIG_NAMES:
-        wl = workloads.make(name)
-        vb = workloads.valid_bytes(wl.lengths)
-        tensor_bytes = wl.logits.nbytes
-        R = max(1, min(64, -(-4 * L2_BYTES // tensor_bytes)))
-        base = torch.from_numpy(wl.logits).cuda()
-        copies = [base] + [base.clone() for _ in range(R - 1)]
-        lengths = torch.from_numpy(wl.lengths).cuda()
-        out = torch.empty((wl.num_rows, wl.k), dtype=torch.int32, device="cuda")
-        n_calls = max(R, min(256, max(8, int(2e9 // max(vb, 1)))))
-        cold = [(lambda c=copies[i % R]: dsa.dsa_topk(c, lengths, wl.k, out=out)) for i in range(n_calls)]
-        us_cold = time_graph(dsa, torch, cold)
-        warm = [(lambda: dsa.dsa_topk(base, lengths, wl.k, out=out)) for _ in range(min(n_calls, 64))]
-        us_warm = time_graph(dsa, torch, warm)
-        cs, grid = dsa.plan(wl.num_rows, wl.row_stride, wl.k)
-        gbs = vb / us_cold / 1e3
-        rows[name] = {
-            "us_per_call": round(us_cold, 3), "rows_per_s": round(wl.num_rows / us_cold * 1e6, 1),
-            "valid_gbs": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
-            "us_per_call_warm_l2": round(us_warm, 3), "valid_bytes": vb,
-            "rotating_copies": R, "cluster_size": cs, "grid": grid,
-        }
-        del copies, base, out
-        torch.cuda.empty_cache()
+        rows[name] = _time_workload(dsa, torch, peak, workloads.make(name))
+    wl = workloads.make("prefill")
+    rows["prefill_bf16"] = _time_workload(dsa, torch, peak, wl, dtype=torch.bfloat16)
+    rows["prefill_unsorted"] = _time_workload(dsa, torch, peak, wl, unsorted=True)
+    rows["prefill_index_table"] = _time_workload(dsa, torch, peak, wl, table=True)
     return rows
 
 
@@ -264,7 +293,13 @@ def run_ours(args):
     import sparse_attention_indexer_strided_b200 as dsa
 
     peak, peak_src = load_peaks()
-    wl = load_workload(args.config, args.rows)
+    if args.shard == "rows":
+        from sparse_attention_indexer_strided_b200 import shard
+        batch_rows = args.rows or workloads.spec(args.config).num_rows
+        r0, r1 = shard.row_block(batch_rows, world, rank)
+        wl = workloads.make_rows(args.config, range(r0, r1))  # this rank's rows only
+    else:
+        wl = load_workload(args.config, args.rows)
     vb = workloads.valid_bytes(wl.lengths)
     logits = torch.from_numpy(wl.logits).cuda()
     lengths = torch.from_numpy(wl.lengths).cuda()
@@ -298,20 +333,27 @@ def run_ours(args):
     # ---- end to end through the host-buffer C-ABI entry point
     e2e = None
     if args.e2e_steps > 0:
-        e2e = run_e2e(args, dsa, torch, dist, wl, logits, lengths, out, stream, world)
+        e2e = run_e2e(args, dsa, torch, dist, wl, logits, lengths, out, stream, world,
+                      batch_rows if args.shard == "rows" else None)
 
     per_launch_us = ms / args.steps * 1e3
     achieved = vb / per_launch_us / 1e3  # GB/s of valid logits
+    if args.shard == "rows":
+        value = sharded_rows_per_s(batch_rows, args.steps, ms_max)
+        parallelism = "rows%d (one batch in contiguous row blocks, no data-path collective)" % world
+    else:
+        value = job_rows_per_s(world, wl.num_rows, args.steps, ms_max)
+        parallelism = "dp%d (each GPU its own batch, no data-path collective)" % world
     result = {
         "metric": METRIC,
-        "value": round(job_rows_per_s(world, wl.num_rows, args.steps, ms_max), 1),
+        "value": round(value, 1),
         "unit": "rows/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms_max / args.steps, 5),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if args.shard == "rows" else "weak",
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
@@ -321,7 +363,7 @@ def run_ours(args):
             "valid_bytes_per_step": vb,
             "l2": ("inputs %.2f GB > 126 MB L2, no flush needed" % (wl.logits.nbytes / 1e9)
                    if wl.logits.nbytes > 4 * L2_BYTES else "inputs smaller than L2: numbers are L2-warm"),
-            "parallelism": "dp%d (each GPU its own batch, no data-path collective)" % world,
+            "parallelism": parallelism,
             "launch": {"cluster_size": cs, "grid": grid},
             "input_sha256_16": workloads.sha256(wl.logits)[:16],
         },
@@ -350,9 +392,11 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
-def run_e2e(args, dsa, torch, dist, wl, logits, lengths, out, stream, world):
+def run_e2e(args, dsa, torch, dist, wl, logits, lengths, out, stream, world, batch_rows=None):
     """Same metric through dsa_topk_host: pinned host inputs copied in and the
-    result copied out inside the timed region, every step."""
+    result copied out inside the timed region, every step. ``batch_rows``: row
+    shards of one batch (rows/s of that batch); None: one batch per rank.
+    Bytes per step are whole-job figures (all ranks)."""
     h_logits = torch.from_numpy(wl.logits).pin_memory()
     h_len = torch.from_numpy(wl.lengths).pin_memory()
     h_out = torch.empty((wl.num_rows, wl.k), dtype=torch.int32).pin_memory()
@@ -371,11 +415,15 @@ def run_e2e(args, dsa, torch, dist, wl, logits, lengths, out, stream, world):
     e2e_ms = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device="cuda")
     if world > 1:
         dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    value = world * wl.num_rows * args.e2e_steps / (float(e2e_ms.item()) / 1e3)
-    return {"value": round(value, 1), "unit": "rows/s",
-            "h2d_bytes_per_step": int(wl.logits.nbytes + wl.lengths.nbytes),
-            "d2h_bytes_per_step": int(wl.num_rows * wl.k * 4), "steps": args.e2e_steps,
-            "api": "dsa_topk_host (C ABI, pinned host buffers)"}
+    sec = float(e2e_ms.item()) / 1e3
+    io = torch.tensor([float(wl.logits.nbytes + wl.lengths.nbytes), float(wl.num_rows * wl.k * 4)],
+                      dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(io, op=dist.ReduceOp.SUM)
+    rows = batch_rows if batch_rows is not None else world * wl.num_rows
+    return {"value": round(rows * args.e2e_steps / sec, 1), "unit": "rows/s",
+            "h2d_bytes_per_step": int(io[0].item()), "d2h_bytes_per_step": int(io[1].item()),
+            "steps": args.e2e_steps, "api": "dsa_topk_host (C ABI, pinned host buffers)"}
 
 
 def oracle_sample_rows(config, n_rows, offset=0):

@@ -33,6 +33,8 @@ _I32 = ctypes.c_int32
 
 _lib.dsa_topk.restype = ctypes.c_int
 _lib.dsa_topk.argtypes = [_P, _I64, _P, _I64, _I32, _P, _P]
+_lib.dsa_topk_ex.restype = ctypes.c_int
+_lib.dsa_topk_ex.argtypes = [_P, _I32, _I64, _P, _I64, _I32, ctypes.c_uint32, _P, _I64, _P, _P]
 _lib.dsa_topk_host.restype = ctypes.c_int
 _lib.dsa_topk_host.argtypes = [_P, _I64, _P, _I64, _I32, _P, _P, _P, _P, _P]
 _lib.dsa_topk_plan.restype = ctypes.c_int
@@ -43,6 +45,17 @@ _lib.dsa_topk_strerror.restype = ctypes.c_char_p
 _lib.dsa_topk_strerror.argtypes = [ctypes.c_int]
 _lib.dsa_topk_version.restype = ctypes.c_int
 _lib.dsa_topk_version.argtypes = []
+_lib.dsa_topk_set_test_hooks.restype = ctypes.c_int
+_lib.dsa_topk_set_test_hooks.argtypes = [ctypes.c_uint64, _I64]
+
+DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
+FLAG_UNSORTED = 1
+_DTYPES = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}
+
+STATUS_WAIT_TIMEOUT = 1
+STATUS_SELECT_BROKEN = 2
+STATUS_REREAD = 4
+STATUS_ERRORS = STATUS_WAIT_TIMEOUT | STATUS_SELECT_BROKEN
 
 lib = _lib  # raw ctypes handle, for callers that pass their own pointers
 
@@ -67,9 +80,9 @@ def _stream_handle(stream) -> int:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def _check_rows(logits: torch.Tensor, lengths: torch.Tensor, k: int) -> Tuple[int, int]:
-    if logits.dtype != torch.float32 or logits.dim() != 2:
-        raise TypeError("logits must be a 2-D float32 tensor")
+def _check_rows(logits: torch.Tensor, lengths: torch.Tensor, k: int, dtypes=(torch.float32,)) -> Tuple[int, int]:
+    if logits.dtype not in dtypes or logits.dim() != 2:
+        raise TypeError("logits must be a 2-D tensor of one of %s" % (dtypes,))
     if logits.size(0) > 0 and logits.size(1) > 1 and logits.stride(1) != 1:
         raise ValueError("logits rows must be contiguous along dim 1 (stride(1) == 1)")
     if lengths.dtype != torch.int32 or lengths.dim() != 1 or lengths.size(0) != logits.size(0):
@@ -88,23 +101,40 @@ def _check_rows(logits: torch.Tensor, lengths: torch.Tensor, k: int) -> Tuple[in
 
 
 def dsa_topk(logits: torch.Tensor, lengths: torch.Tensor, k: int,
-             out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+             out: Optional[torch.Tensor] = None, stream=None, unsorted: bool = False,
+             index_table: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Top-k row-local indices of ``logits[r, :lengths[r]]`` per row.
 
-    ``logits``: CUDA float32 ``[num_rows, >= max L]``, any row stride.
-    ``lengths``: CUDA int32 ``[num_rows]`` (clamped to [0, stride] on device).
-    Returns (or fills ``out``) int32 ``[num_rows, k]``: value descending, ties
-    by ascending index, -1 past ``min(k, L_r)``. Asynchronous on ``stream``.
+    ``logits``: CUDA float32, bfloat16 or float16 ``[num_rows, >= max L]``,
+    any row stride. ``lengths``: CUDA int32 ``[num_rows]`` (clamped to [0,
+    stride] on device). Returns (or fills ``out``) int32 ``[num_rows, k]``:
+    value descending, ties by ascending index, -1 past ``min(k, L_r)``.
+    ``unsorted``: the same index set per row, in unspecified order.
+    ``index_table``: CUDA int32 ``[num_rows, >= max L]`` (any row stride); each
+    selected index j of row r is written as ``index_table[r, j]``.
+    Asynchronous on ``stream``.
     """
-    rows, stride = _check_rows(logits, lengths, k)
+    rows, stride = _check_rows(logits, lengths, k, tuple(_DTYPES))
     if not (logits.is_cuda and lengths.is_cuda):
         raise ValueError("logits and lengths must be CUDA tensors (use dsa_topk_host for host buffers)")
     if out is None:
         out = torch.empty((rows, k), dtype=torch.int32, device=logits.device)
     elif out.dtype != torch.int32 or tuple(out.shape) != (rows, k) or not out.is_contiguous():
         raise ValueError("out must be contiguous int32 [num_rows, k]")
-    rc = _lib.dsa_topk(logits.data_ptr(), stride, lengths.data_ptr(), rows, int(k), out.data_ptr(),
-                       _stream_handle(stream))
+    if logits.dtype == torch.float32 and not unsorted and index_table is None:
+        rc = _lib.dsa_topk(logits.data_ptr(), stride, lengths.data_ptr(), rows, int(k), out.data_ptr(),
+                           _stream_handle(stream))
+    else:
+        tptr, tstride = None, 0
+        if index_table is not None:
+            if (index_table.dtype != torch.int32 or index_table.dim() != 2 or not index_table.is_cuda
+                    or index_table.size(0) != rows or (index_table.size(1) > 1 and index_table.stride(1) != 1)):
+                raise ValueError("index_table must be a CUDA int32 [num_rows, >= max L] tensor with stride(1) == 1")
+            tptr = index_table.data_ptr()
+            tstride = int(index_table.stride(0)) if rows > 1 else max(int(index_table.size(1)), 1)
+        rc = _lib.dsa_topk_ex(logits.data_ptr(), _DTYPES[logits.dtype], stride, lengths.data_ptr(), rows, int(k),
+                              FLAG_UNSORTED if unsorted else 0, tptr, tstride, out.data_ptr(),
+                              _stream_handle(stream))
     if rc != 0:
         raise DsaTopkError(rc)
     return out
@@ -144,7 +174,8 @@ def plan(num_rows: int, row_stride: int, k: int) -> Tuple[int, int]:
 
 
 def device_status(clear: bool = False) -> int:
-    """Sticky device-side status bits (bit 0: a pipeline wait timed out). Syncs."""
+    """Sticky device-side status bits (``STATUS_*``; ``STATUS_ERRORS`` are the
+    error bits, ``STATUS_REREAD`` is informational). Syncs the device."""
     v = ctypes.c_uint32(0)
     rc = _lib.dsa_topk_device_status(ctypes.byref(v), 1 if clear else 0)
     if rc != 0:
@@ -152,5 +183,15 @@ def device_status(clear: bool = False) -> int:
     return int(v.value)
 
 
-__all__ = ["dsa_topk", "dsa_topk_host", "plan", "device_status", "strerror", "version",
-           "DsaTopkError", "MAX_K", "LIB_PATH", "lib"]
+def set_test_hooks(wait_limit_ns: int = 0, skip_stage: int = -1) -> None:
+    """Test use only: the time limit of every device-side wait (0: default
+    0.5 s) and a stage each CTA's producer leaves unissued (-1: none)."""
+    rc = _lib.dsa_topk_set_test_hooks(int(wait_limit_ns), int(skip_stage))
+    if rc != 0:
+        raise DsaTopkError(rc)
+
+
+__all__ = ["dsa_topk", "dsa_topk_host", "plan", "device_status", "set_test_hooks", "strerror", "version",
+           "DTYPE_F32", "DTYPE_BF16", "DTYPE_F16", "FLAG_UNSORTED",
+           "DsaTopkError", "MAX_K", "LIB_PATH", "lib", "STATUS_WAIT_TIMEOUT", "STATUS_SELECT_BROKEN",
+           "STATUS_REREAD", "STATUS_ERRORS"]

@@ -1,0 +1,1477 @@
+// The top-k kernel: one persistent CTA per SM over many rows, or a
+// thread-block cluster per row when rows are few and long.
+//
+// Many-row mode (cluster size 1, 480 threads, three warp roles):
+//   producer (1 warp, one lane)  : cp.async.bulk copies of the CTA's rows, in
+//                                  8192-element stages, into a 96 KB shared
+//                                  ring (full / empty mbarriers).
+//   filter   (8 warps)           : every stage, each lane compares its 32
+//                                  values with the row's running threshold t
+//                                  (keep x unless x < t; NaN always kept); the
+//                                  warps meet at one barrier per stage to place
+//                                  the survivors' (key, index) pairs in a
+//                                  shared candidate buffer. Once m candidates
+//                                  at or above t are held, t becomes strict (a
+//                                  later equal value has a larger index, so it
+//                                  loses its tie). When the buffer passes half
+//                                  full it is compacted: an approximate radix
+//                                  cut when one suffices, else an exact select
+//                                  with the tie cut by index. At the end of the
+//                                  row the candidates are handed over.
+//   finisher (6 warps)           : ranks the handed-over candidates by (key
+//                                  descending, index ascending) with bucket
+//                                  passes over a composite key (a bitonic sort
+//                                  when a bucket stays crowded with equal
+//                                  keys), then writes the first m indices and
+//                                  -1 padding while the filter warps already
+//                                  stream the next row.
+//
+// A row starts with a speculative threshold: from the row the finisher
+// completed two rows earlier (half the gap between that row's 3k/4-th and
+// k-th largest below its k-th), else from the threshold that passed enough of
+// the CTA's previous row, else from a sample of the row itself. If fewer than
+// m values pass it, the filter warps re-read the row from global memory with
+// no threshold; the result is exact either way, only the time changes.
+//
+// Cluster mode (a cluster of C CTAs per row, 288 threads: filter warps and a
+// producer warp, no finisher warps): rank r streams the contiguous chunk r of
+// the row exactly as a row is streamed above, keeping a superset of the
+// chunk's top min(m, chunk). The ranks then merge through distributed shared
+// memory (SGLang PR #34167 code excerpt, TopKCluster::forward: per-rank
+// counts, cluster barriers between phases, rank-ordered write offsets):
+// counts and key bounds are published, cluster-wide histogram rounds narrow a
+// threshold until the survivors fit the leader's buffer, and every rank writes
+// its survivors into the leader's shared memory at rank-ordered offsets (a
+// tied threshold value is shared out in rank order, which is index order).
+// The leader's filter warps then rank and write the row like the finisher.
+// DSMEM addresses are 32-bit shared::cluster addresses used only with
+// ld/st.shared::cluster (the SGLang page traces a miscompile to merging them
+// with CTA pointers).
+//
+// The selection follows the pages' histogram / cumulative-sum / threshold /
+// gt-eq split (SGLang PR #34167 code excerpt, the radix top-k kernel), made
+// exact: ties at the threshold go to the lowest indices (a second radix select
+// over the indices of the tied keys) instead of a capped tie list.
+#pragma once
+
+#include "common.cuh"
+
+namespace dsa {
+namespace rows {
+
+constexpr int kFilterWarps = 8;
+constexpr int kFilterThreads = kFilterWarps * 32;  // 256
+constexpr int kFinishWarps = 6;
+constexpr int kFinishThreads = kFinishWarps * 32;  // 192
+constexpr int kProducerWarp = kFilterWarps + kFinishWarps;
+constexpr int kThreads = (kProducerWarp + 1) * 32;      // 480: many-row mode
+constexpr int kClusterWarp = kFilterWarps;              // cluster mode: the producer warp
+constexpr int kClusterThreads = (kFilterWarps + 1) * 32;  // 288: cluster mode
+constexpr int kGroups = 8;                              // groups of 4 values per lane and stage
+constexpr int kVals = 4 * kGroups;                      // 32 values per lane and stage
+constexpr int kWarpElems = 32 * kVals;                  // 1024 per warp and stage
+constexpr int kStageElems = kFilterWarps * kWarpElems;  // 8192
+constexpr int kRingBytes = 3 * 32768;                   // 96 KB ring
+constexpr int kMaxStages = 6;
+constexpr int kFiltCap = 8192;                          // candidate buffer entries
+constexpr int kTrigger = kFiltCap / 2;                  // compact after a stage that leaves more
+constexpr int kHandCap = 4096;                          // handed-over (or gathered) candidates, at most
+constexpr int kPerThread = (kFiltCap + kFilterThreads - 1) / kFilterThreads;  // entries per filter thread
+constexpr int kRounds = 4;                              // radix rounds of 8 bits
+constexpr int kKeepLimit = 2560;                        // approximate compaction keeps at most this many
+constexpr int kSampleRunsPerWarp = 4;                   // runs of 128 each filter warp samples
+constexpr int kSampleChunks = kFilterWarps * kSampleRunsPerWarp;  // runs sampled for a row's first threshold
+constexpr int kSampleVals = kSampleChunks * 128;        // 4096 sampled values
+constexpr int64_t kSampleMinLen = 4 * kStageElems;      // shorter rows start with no threshold
+constexpr int kBigBucket = 64;                          // finisher: larger buckets are sorted instead
+constexpr int kSmallBucket = 16;                        // finisher: largest bucket ranked by direct counting
+constexpr int kSortPasses = 3;                          // finisher: bucket count passes, at most
+constexpr int kBucketMax = 4096;                        // finisher bucket counters
+constexpr uint32_t kAbortBit = 0x80000000u;             // flag bit beside a published stage count
+constexpr uint32_t kUnsorted = DSA_FLAG_UNSORTED;
+
+template <class T>
+__host__ __device__ constexpr int stages_of() {
+  return kRingBytes / (kStageElems * static_cast<int>(sizeof(T)));
+}
+
+static_assert(kVals <= 32, "a lane's survivors of one stage form a 32-bit mask");
+static_assert(kFiltCap - kTrigger >= kStageElems / 2, "half a stage fits after a compaction");
+static_assert(kFilterWarps % 2 == 0 && kKeepLimit + kStageElems / 2 <= kFiltCap, "split halves fit after a compaction");
+static_assert(kHandCap >= kMaxK && kTrigger >= kMaxK, "buffers must hold k entries");
+static_assert(stages_of<float>() == 3 && stages_of<__half>() == 6 && stages_of<__half>() <= kMaxStages, "ring");
+
+// Call parameters (the C ABI's arguments).
+struct Params {
+  const void* logits;
+  int64_t row_stride;  // elements
+  const int32_t* lengths;
+  int64_t num_rows;
+  int32_t k;
+  uint32_t flags;        // DSA_FLAG_*
+  const int32_t* table;  // optional index table: out = table[row * table_stride + idx]
+  int64_t table_stride;
+  int32_t* out;
+};
+
+struct __align__(128) Smem {
+  unsigned char ring[kRingBytes];  // stages of kStageElems elements
+  uint32_t fkey[kFiltCap];         // filter candidates
+  uint32_t fidx[kFiltCap];
+  uint32_t hkey[kHandCap];  // handed over to the finishers (cluster mode: gathered at the leader)
+  uint32_t hidx[kHandCap];
+  uint32_t bcnt[kBucketMax];  // finisher bucket counters / ends (cluster mode: merge histograms first)
+  uint16_t perm[kHandCap];    // finisher: candidates grouped by bucket
+  int32_t ostage[kMaxK];      // finisher: the row's output, written out coalesced
+  uint32_t hist[256];         // filter radix histogram
+  uint4 red[2][(kFilterWarps + 3) / 4];  // per-warp survivor counts, by stage parity
+  uint32_t fred[4][kFilterWarps];
+  uint32_t nred[5][kFilterWarps];  // finisher per-warp reductions (6 or 8 warps)
+  uint32_t bc[8];
+  uint32_t small[32];
+  uint32_t rec[2];  // finisher: keys at ranks k-1 and 3k/4-1
+  uint32_t pub[8];  // cluster mode: published to the other ranks
+  // handover (filter -> finisher)
+  int64_t h_row, h_len;
+  int32_t h_n, h_m;
+  // speculative threshold (finisher -> filter), by handover parity
+  int64_t est_len[2];
+  float est[2];
+  int32_t est_ok[2];
+  // the filter warps' own estimate: an earlier row of length own_len passed at
+  // least k values at or above own_key (own_len 0: none yet)
+  uint32_t own_key;
+  int32_t own_len;
+  float row_t0;        // the current row's initial threshold
+  uint32_t abort;      // raised by the first pipeline wait that gives up
+  uint32_t abort_any;  // cluster mode: some rank gave up (read by the leader)
+  uint32_t final_bar;  // cluster mode: number of cluster barriers of the merge (0: not yet known)
+  unsigned long long full[kMaxStages], empty[kMaxStages];
+  unsigned long long hfull, hempty;
+};
+static_assert(sizeof(Smem) <= 232448, "shared memory budget of one CTA per SM");
+static_assert(2 * 256 + 256 <= kBucketMax, "merge histograms alias the bucket counters");
+
+__device__ __forceinline__ void bar_filter() { asm volatile("bar.sync 1, %0;" ::"n"(kFilterThreads) : "memory"); }
+// Named barrier that also returns whether any participating thread passed
+// true: every thread of the role takes the same branch afterwards.
+template <int kBar, int kCount>
+__device__ __forceinline__ bool bar_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "n"(kBar), "n"(kCount)
+      : "memory");
+  return r != 0u;
+}
+__device__ __forceinline__ bool bar_filter_any(bool pred) { return bar_any<1, kFilterThreads>(pred); }
+
+// Smallest float threshold t with (!(x < t)) == (key(x) > T) for every non-NaN x.
+// T at or above +inf's key has no such float: +inf is returned, which also
+// keeps +inf itself (a superset, harmless: the final ranking is exact).
+__device__ __forceinline__ float above(uint32_t T) {
+  return T < kInfKey ? from_key(T + 1u) : __int_as_float(0x7f800000);
+}
+
+// The 16-byte aligned byte span covering item entries [0, L) of an item that
+// starts at element pointer `row`.
+struct RowSpan {
+  const char* src;
+  int64_t j0;           // item index of the span's first element (-7..0)
+  int nst;              // stages
+  uint32_t last_bytes;  // bytes of the last stage
+};
+
+template <class T>
+__device__ __forceinline__ RowSpan row_span(const T* row, int64_t L) {
+  constexpr uint32_t kStageBytes = kStageElems * sizeof(T);
+  RowSpan sp;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(row);
+  const uintptr_t as = a & ~static_cast<uintptr_t>(15);
+  sp.src = reinterpret_cast<const char*>(as);
+  sp.j0 = -static_cast<int64_t>((a - as) / sizeof(T));
+  if (L <= 0) {
+    sp.nst = 0;
+    sp.last_bytes = 0;
+    return sp;
+  }
+  const uintptr_t ee = (reinterpret_cast<uintptr_t>(row + L) + 15) & ~static_cast<uintptr_t>(15);
+  const uint64_t bytes = ee - as;
+  sp.nst = static_cast<int>((bytes + kStageBytes - 1) / kStageBytes);
+  sp.last_bytes = static_cast<uint32_t>(bytes - static_cast<uint64_t>(sp.nst - 1) * kStageBytes);
+  return sp;
+}
+
+// ------------------------------------------------------------ filter warps
+// Position of value j (0..31) of a lane inside its stage: group j/4 of four
+// consecutive elements at warp*kWarpElems + (j/4)*128 + lane*4 (conflict-free
+// 128-bit (fp32) or 64-bit (16-bit types) shared loads).
+__device__ __forceinline__ int val_offset(int w, int lane, int j) {
+  return w * kWarpElems + (j >> 2) * 128 + lane * 4 + (j & 3);
+}
+
+__device__ __forceinline__ uint32_t pass_mask(const float (&v)[kVals], float t) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < kVals; ++j) m |= static_cast<uint32_t>(!(v[j] < t)) << j;
+  return m;
+}
+
+// Stage-local offsets [lo, hi) of a stage whose first element has item index
+// sj0 that hold item indices in [0, L).
+__device__ __forceinline__ void stage_bounds(int64_t sj0, int64_t L, int& lo, int& hi) {
+  const int64_t a = -sj0, b = L - sj0;
+  lo = static_cast<int>(a < 0 ? 0 : (a > kStageElems ? kStageElems : a));
+  hi = static_cast<int>(b < 0 ? 0 : (b > kStageElems ? kStageElems : b));
+}
+
+// Bits of this lane's values whose stage offset lies in [lo, hi).
+__device__ __forceinline__ uint32_t range_mask(int w, int lane, int lo, int hi) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < kVals; ++j) {
+    const int o = val_offset(w, lane, j);
+    m |= static_cast<uint32_t>(o >= lo && o < hi) << j;
+  }
+  return m;
+}
+
+// min / max of v(e) over candidates [0, n) with pred(e) (filter threads).
+template <class V, class P>
+__device__ void filter_minmax(Smem& s, int n, V v, P pred, uint32_t& lo, uint32_t& hi, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+  for (int e = tid; e < n; e += kFilterThreads) {
+    if (!pred(e)) continue;
+    const uint32_t x = v(e);
+    mn = min(mn, x);
+    mx = max(mx, x);
+  }
+  mn = __reduce_min_sync(kFull, mn);
+  mx = __reduce_max_sync(kFull, mx);
+  if (lane == 0) {
+    s.fred[0][w] = mn;
+    s.fred[1][w] = mx;
+  }
+  bar_filter();
+  lo = __reduce_min_sync(kFull, lane < kFilterWarps ? s.fred[0][lane] : 0xFFFFFFFFu);
+  hi = __reduce_max_sync(kFull, lane < kFilterWarps ? s.fred[1][lane] : 0u);
+  bar_filter();
+}
+
+// 256-bin histogram of the 8-bit digit at bit sh of v(e), over the entries
+// [0, n) with pred(e) and v(e) in [lo, hi] (hist zeroed, filter threads).
+// Lanes of a warp holding the same digit are merged first (match.any), so
+// one atomic per distinct digit and warp: values on a few levels (ties, the
+// top byte of floats of one sign) would otherwise queue thousands of atomics
+// on one counter.
+template <class V, class P>
+__device__ __forceinline__ void digit_histogram(uint32_t* hist, int n, V v, P pred, uint32_t lo, uint32_t hi, int sh,
+                                                int tid) {
+  const uint32_t lt = lanemask_lt();
+  for (int e0 = 0; e0 < n; e0 += kFilterThreads) {  // warp-uniform trip count
+    const int e = e0 + tid;
+    uint32_t d = 0xFFFFFFFFu;
+    if (e < n && pred(e)) {
+      const uint32_t x = v(e);
+      if (x >= lo && x <= hi) d = (x >> sh) & 255u;
+    }
+    const uint32_t peers = __match_any_sync(kFull, d);
+    if (d != 0xFFFFFFFFu && (peers & lt) == 0u) atomicAdd(&hist[d], __popc(peers));
+  }
+}
+
+// need-th largest of v(e) over the candidates with pred(e) (1 <= need <= their
+// number). Radix rounds over 8-bit windows below the highest bit where the
+// bounds differ; after each round the bounds shrink to the smallest and
+// largest value actually inside the chosen bucket (a bucket of one tied value
+// ends the search there). A bucket of <= 32 values is finished by one warp.
+template <class V, class P>
+__device__ uint32_t filter_kth(Smem& s, int n, uint32_t need, V v, P pred, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  uint32_t lo, hi;
+  filter_minmax(s, n, v, pred, lo, hi, tid);
+  for (int round = 0; lo != hi; ++round) {
+    if (round == kRounds) {  // unreachable for a consistent histogram
+      if (tid == 0) atomicOr(&g_status, kStatusSelectBroken);
+      break;
+    }
+    const int sh = window_shift(lo, hi);
+    for (int i = tid; i < 256; i += kFilterThreads) s.hist[i] = 0u;
+    if (tid == 0) {
+      s.bc[0] = 0xFFFFFFFFu;
+      s.bc[2] = 0u;
+    }
+    bar_filter();
+    digit_histogram(s.hist, n, v, pred, lo, hi, sh, tid);
+    bar_filter();
+    if (w == 0) find_bucket_warp0(s.hist, need, s.bc, lane);
+    bar_filter();
+    const uint32_t bsel = s.bc[0], above_b = s.bc[1];
+    if (bsel == 0xFFFFFFFFu) {
+      if (tid == 0) atomicOr(&g_status, kStatusSelectBroken);
+      break;
+    }
+    const uint32_t in_bucket = s.hist[bsel];
+    need -= above_b;
+    narrow(lo, hi, sh, bsel);
+    if (in_bucket <= 32u && lo != hi) {
+      for (int e = tid; e < n; e += kFilterThreads) {
+        if (!pred(e)) continue;
+        const uint32_t x = v(e);
+        if (x >= lo && x <= hi) {
+          const uint32_t slot = atomicAdd(&s.bc[2], 1u);
+          if (slot < 32u) s.small[slot] = x;
+        }
+      }
+      bar_filter();
+      if (w == 0) {
+        const uint32_t t = small_kth(lane < static_cast<int>(in_bucket) ? s.small[lane] : 0u, need);
+        if (lane == 0) s.bc[3] = t;
+      }
+      bar_filter();
+      lo = hi = s.bc[3];
+    } else if (lo != hi) {
+      const uint32_t a = lo, b = hi;
+      filter_minmax(s, n, v, [&](int e) { return pred(e) && v(e) >= a && v(e) <= b; }, lo, hi, tid);
+    }
+    bar_filter();
+  }
+  return lo;
+}
+
+struct FKey {
+  const Smem* s;
+  __device__ uint32_t operator()(int e) const { return s->fkey[e]; }
+};
+struct FNotIdx {  // larger value = smaller index
+  const Smem* s;
+  __device__ uint32_t operator()(int e) const { return ~s->fidx[e]; }
+};
+struct FAll {
+  __device__ bool operator()(int) const { return true; }
+};
+struct FKeyIs {
+  const Smem* s;
+  uint32_t T;
+  __device__ bool operator()(int e) const { return s->fkey[e] == T; }
+};
+
+// Keeps the candidates with key > A and, when kTies, those with key == A and
+// index <= I: in place and in any order (local), or stored at positions
+// off.. of the shared::cluster addresses rkey / ridx (remote, cluster mode).
+// Every filter thread reads its entries before any is written. Returns the
+// kept count (uniform).
+template <bool kTies, bool kRemote = false>
+__device__ uint32_t keep_pass(Smem& s, int n, uint32_t A, uint32_t I, int tid, uint32_t rkey = 0u, uint32_t ridx = 0u,
+                              uint32_t off = 0u) {
+  const int w = tid >> 5, lane = tid & 31;
+  uint32_t kk[kPerThread], ii[kPerThread], keep = 0;
+#pragma unroll
+  for (int it = 0; it < kPerThread; ++it) {
+    const int e = it * kFilterThreads + tid;
+    kk[it] = 0u;
+    ii[it] = 0u;
+    if (e < n) {
+      kk[it] = s.fkey[e];
+      ii[it] = s.fidx[e];
+    }
+    const bool kp = e < n && (kk[it] > A || (kTies && kk[it] == A && ii[it] <= I));
+    keep |= static_cast<uint32_t>(kp) << it;
+  }
+  const uint32_t nk = __popc(keep);
+  uint32_t incl = nk;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) s.fred[0][w] = incl;
+  bar_filter();
+  uint32_t pos = incl - nk, total = 0;
+#pragma unroll
+  for (int ww = 0; ww < kFilterWarps; ++ww) {
+    const uint32_t c = s.fred[0][ww];
+    pos += ww < w ? c : 0u;
+    total += c;
+  }
+#pragma unroll
+  for (int it = 0; it < kPerThread; ++it) {
+    if ((keep >> it) & 1u) {
+      if (kRemote) {
+        dsmem_st(rkey + 4u * (off + pos), kk[it]);
+        dsmem_st(ridx + 4u * (off + pos), ii[it]);
+      } else {
+        s.fkey[pos] = kk[it];
+        s.fidx[pos] = ii[it];
+      }
+      ++pos;
+    }
+  }
+  bar_filter();
+  return total;
+}
+
+// Index cut among the candidates with key == T: the need-th smallest index
+// (1 <= need <= their number).
+__device__ __forceinline__ uint32_t tie_cut(Smem& s, int n, uint32_t T, uint32_t need, int tid) {
+  return ~filter_kth(s, n, need, FNotIdx{&s}, FKeyIs{&s, T}, tid);
+}
+
+// Counts of candidates [0, n) with key > T and key == T (uniform).
+__device__ void count_gt_eq(Smem& s, int n, uint32_t T, uint32_t& ngt, uint32_t& neq, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  uint32_t g = 0, q = 0;
+  for (int e = tid; e < n; e += kFilterThreads) {
+    const uint32_t key = s.fkey[e];
+    g += key > T;
+    q += key == T;
+  }
+  g = __reduce_add_sync(kFull, g);
+  q = __reduce_add_sync(kFull, q);
+  if (lane == 0) {
+    s.fred[2][w] = g;
+    s.fred[3][w] = q;
+  }
+  bar_filter();
+  ngt = __reduce_add_sync(kFull, lane < kFilterWarps ? s.fred[2][lane] : 0u);
+  neq = __reduce_add_sync(kFull, lane < kFilterWarps ? s.fred[3][lane] : 0u);
+  bar_filter();
+}
+
+// Exact: keeps the top m of candidates [0, n) by (key descending, index
+// ascending), n > m >= 1. Returns the m-th largest key.
+__device__ __noinline__ uint32_t compact_exact(Smem& s, int n, int m, int tid) {
+  bar_filter();  // every append is visible
+  const uint32_t T = filter_kth(s, n, static_cast<uint32_t>(m), FKey{&s}, FAll{}, tid);
+  uint32_t ngt, neq;
+  count_gt_eq(s, n, T, ngt, neq, tid);
+  const uint32_t need = static_cast<uint32_t>(m) - ngt;  // entries equal to T that stay
+  uint32_t I = 0xFFFFFFFFu;                               // largest index of a kept tie
+  if (neq > need) I = tie_cut(s, n, T, need, tid);
+  keep_pass<true>(s, n, T, I, tid);
+  return T;
+}
+
+// Approximate: narrows the radix bucket holding the m-th largest key until
+// every key at or above the bucket's lower end fits in kKeepLimit entries,
+// then keeps exactly those (a superset of the top m). Returns ok = 0, having
+// changed nothing, when that needs more than kRounds rounds or the bucket is
+// one tied key with too many entries: the exact pass must run.
+struct FastCut {
+  uint32_t ok, lo, kept;
+};
+
+__device__ __noinline__ FastCut compact_fast(Smem& s, int n, int m, int tid) {
+  uint32_t kept = 0;
+  const int w = tid >> 5, lane = tid & 31;
+  bar_filter();  // every append is visible
+  uint32_t lo, hi;
+  filter_minmax(s, n, FKey{&s}, FAll{}, lo, hi, tid);
+  uint32_t need = static_cast<uint32_t>(m), above_lo = 0;
+  bool ok = false;
+  for (int round = 0; round < kRounds && lo != hi; ++round) {
+    const int sh = window_shift(lo, hi);
+    for (int i = tid; i < 256; i += kFilterThreads) s.hist[i] = 0u;
+    if (tid == 0) s.bc[0] = 0xFFFFFFFFu;
+    bar_filter();
+    digit_histogram(s.hist, n, FKey{&s}, FAll{}, lo, hi, sh, tid);
+    bar_filter();
+    if (w == 0) find_bucket_warp0(s.hist, need, s.bc, lane);
+    bar_filter();
+    const uint32_t bsel = s.bc[0];
+    const uint32_t above_b = s.bc[1];
+    const uint32_t in_b = bsel == 0xFFFFFFFFu ? 0u : s.hist[bsel];
+    bar_filter();  // hist and bc are rewritten by the next round
+    if (bsel == 0xFFFFFFFFu) {
+      if (tid == 0) atomicOr(&g_status, kStatusSelectBroken);
+      break;
+    }
+    above_lo += above_b;
+    need -= above_b;
+    narrow(lo, hi, sh, bsel);
+    if (above_lo + in_b <= static_cast<uint32_t>(kKeepLimit)) {
+      ok = true;
+      kept = above_lo + in_b;
+      break;
+    }
+  }
+  if (!ok) return FastCut{0u, 0u, 0u};
+  keep_pass<false>(s, n, lo - 1u, 0u, tid);  // key >= lo (every real key is >= 1)
+  return FastCut{1u, lo, kept};
+}
+
+struct Filter {
+  uint32_t cnt;       // candidates held (the same in every filter thread)
+  float t;            // keep x unless x < t
+  int par;            // stage parity of s.red on the synchronous path
+  bool compacted;     // the item was compacted at least once
+  bool strict;        // t already excludes values equal to the held m-th key
+  bool bounded;       // last_key is set
+  uint32_t last_key;  // at least m candidates with key >= last_key are held
+};
+
+// Holding at least m candidates, every one at or above the threshold t: a
+// later value equal to t has a larger index than all of them and cannot enter
+// the top m, so the threshold becomes strict (rows of tied values then stop
+// filling the buffer).
+__device__ __forceinline__ void tighten(Filter& f, int m) {
+  if (!f.strict && m > 0 && f.cnt >= static_cast<uint32_t>(m)) {
+    f.last_key = to_key(f.t);
+    f.bounded = true;
+    f.t = above(f.last_key);
+    f.strict = true;
+  }
+}
+
+// Bounds the buffer again: the approximate pass, else the exact one.
+__device__ __forceinline__ void compact_any(Smem& s, Filter& f, int m, int tid) {
+  const FastCut c = compact_fast(s, static_cast<int>(f.cnt), m, tid);
+  if (c.ok) {
+    f.cnt = c.kept;
+    f.t = c.lo > kInfKey ? __int_as_float(0x7f800000) : from_key(c.lo);
+    f.last_key = c.lo;
+    f.bounded = true;
+    f.strict = false;
+    tighten(f, m);
+  } else {
+    const uint32_t T = compact_exact(s, static_cast<int>(f.cnt), m, tid);
+    f.cnt = static_cast<uint32_t>(m);
+    f.t = above(T);
+    f.last_key = T;
+    f.bounded = true;
+    f.strict = true;
+  }
+  f.compacted = true;
+}
+
+// Writes this warp's survivors (bit j of msk: value j of the lane; values
+// re-read from src, the stage in the ring or in global memory) at positions
+// pos.., up to two survivors per lane and round.
+template <class T, bool kRing>
+__device__ __forceinline__ void put_survivors(Smem& s, const T* src, uint32_t msk, uint32_t idx0, uint32_t pos, int w,
+                                              int lane) {
+  const uint32_t lt = lanemask_lt();
+  uint32_t rest = msk;
+  for (;;) {  // two survivors per lane and iteration: their loads overlap
+    const bool a1 = rest != 0u;
+    const uint32_t b1 = __ballot_sync(kFull, a1);
+    if (b1 == 0u) break;
+    const int j1 = __ffs(rest) - 1;
+    rest &= rest - 1u;
+    const bool a2 = rest != 0u;
+    const uint32_t b2 = __ballot_sync(kFull, a2);
+    const int j2 = __ffs(rest) - 1;
+    rest &= rest - 1u;
+    const uint32_t n1 = __popc(b1);
+    const int o1 = val_offset(w, lane, j1 & 31), o2 = val_offset(w, lane, j2 & 31);
+    float x1 = 0.f, x2 = 0.f;
+    if (a1) x1 = kRing ? Elem<T>::f(src[o1]) : Elem<T>::one_ldg(src + o1);
+    if (a2) x2 = kRing ? Elem<T>::f(src[o2]) : Elem<T>::one_ldg(src + o2);
+    if (a1) {
+      const uint32_t p = pos + __popc(b1 & lt);
+      s.fkey[p] = to_key(x1);
+      s.fidx[p] = idx0 + static_cast<uint32_t>(o1);
+    }
+    if (a2) {
+      const uint32_t p = pos + n1 + __popc(b2 & lt);
+      s.fkey[p] = to_key(x2);
+      s.fidx[p] = idx0 + static_cast<uint32_t>(o2);
+    }
+    pos += n1 + __popc(b2);
+  }
+}
+
+// A stage whose survivors do not fit behind the buffer's contents (rare: no
+// usable threshold yet, or values rising along the row): the warps write in
+// two halves, compacting first whenever a half would not fit. A half with
+// more than the free space implies more than kTrigger >= m entries held, so
+// the compaction applies; afterwards a half (<= kStageElems / 2) fits. Masks
+// taken before a compaction are supersets of the current ones, which is
+// harmless: the final ranking is exact.
+// (Rare paths take and return the filter state by value so that it never has
+// an address and stays in registers in the hot loop. This one and the re-read
+// below are inlined: a real call inside the row loop made the compiler keep
+// loop state in local memory, reloaded on every stage.)
+template <class T, bool kRing>
+__device__ __forceinline__ Filter take_stage_split(Smem& s, Filter f, const uint32_t* red, const T* src, uint32_t msk,
+                                                   uint32_t idx0, int m, int tid) {
+  constexpr int kHalf = kFilterWarps / 2;
+  const int w = tid >> 5, lane = tid & 31;
+  for (int half = 0; half < 2; ++half) {
+    uint32_t tot = 0, before = 0;
+#pragma unroll
+    for (int i = 0; i < kHalf; ++i) {
+      const int ww = kHalf * half + i;
+      const uint32_t c = red[ww];
+      tot += c;
+      before += ww < w ? c : 0u;
+    }
+    if (f.cnt + tot > static_cast<uint32_t>(kFiltCap)) compact_any(s, f, m, tid);
+    if (w / kHalf == half) put_survivors<T, kRing>(s, src, msk, idx0, f.cnt + before, w, lane);
+    f.cnt += tot;
+    bar_filter();  // this half's entries are visible to a following compaction
+  }
+  return f;
+}
+
+// Takes one stage after the filter barrier that completed its per-warp counts.
+// Returns false, writing nothing, when a warp flagged that its wait for the
+// stage gave up (kAbortBit of its count): every filter warp sees the same
+// counts, so all of them leave together.
+template <class T, bool kRing>
+__device__ __forceinline__ bool take_stage(Smem& s, Filter& f, const uint4* red, const T* src, uint32_t msk,
+                                           uint32_t idx0, int m, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  uint32_t r[4 * ((kFilterWarps + 3) / 4)];
+#pragma unroll
+  for (int i = 0; i < (kFilterWarps + 3) / 4; ++i) {
+    const uint4 q = red[i];
+    r[4 * i + 0] = q.x;
+    r[4 * i + 1] = q.y;
+    r[4 * i + 2] = q.z;
+    r[4 * i + 3] = q.w;
+  }
+  uint32_t before = 0, tot = 0, flags = 0;
+#pragma unroll
+  for (int i = 0; i < kFilterWarps; ++i) {
+    before += i < w ? r[i] : 0u;
+    tot += r[i];
+    flags |= r[i];
+  }
+  if (flags & kAbortBit) return false;
+  if (f.cnt + tot <= static_cast<uint32_t>(kFiltCap)) {
+    put_survivors<T, kRing>(s, src, msk, idx0, f.cnt + before, w, lane);
+    f.cnt += tot;
+  } else {
+    f = take_stage_split<T, kRing>(s, f, reinterpret_cast<const uint32_t*>(red), src, msk, idx0, m, tid);
+  }
+  return true;
+}
+
+// Publishes this warp's survivor count (read after the next filter barrier),
+// with kAbortBit set when a lane's wait for the stage gave up.
+__device__ __forceinline__ void publish(uint4* red, uint32_t msk, int w, int lane, bool fail) {
+  const uint32_t wt = __reduce_add_sync(kFull, __popc(msk));
+  const bool ab = __any_sync(kFull, fail);
+  if (lane == 0) reinterpret_cast<uint32_t*>(red)[w] = wt | (ab ? kAbortBit : 0u);
+}
+
+__device__ __forceinline__ uint32_t stage_mask(const float (&v)[kVals], float t, bool edge, int64_t sj0, int64_t L,
+                                               int w, int lane) {
+  uint32_t msk = pass_mask(v, t);
+  if (edge) {
+    int lo, hi;
+    stage_bounds(sj0, L, lo, hi);
+    msk &= range_mask(w, lane, lo, hi);
+  }
+  return msk;
+}
+
+// The speculative threshold let fewer than m values through: stream the item
+// again from global memory with no threshold (one filter barrier per stage).
+template <class T>
+__device__ __forceinline__ Filter refilter_from_global(Smem& s, Filter f, RowSpan sp, int64_t L, uint32_t base, int m,
+                                                       int tid) {
+  constexpr uint32_t kStageBytes = kStageElems * sizeof(T);
+  const int w = tid >> 5, lane = tid & 31;
+  f.cnt = 0;
+  f.t = __int_as_float(0xff800000);  // -inf: keep everything
+  f.compacted = false;
+  f.strict = false;
+  f.bounded = false;
+  for (int st = 0; st < sp.nst; ++st) {
+    const T* src = reinterpret_cast<const T*>(sp.src + static_cast<uint64_t>(st) * kStageBytes);
+    const uint32_t avail = st + 1 == sp.nst ? sp.last_bytes : kStageBytes;
+    const int64_t sj0 = sp.j0 + static_cast<int64_t>(st) * kStageElems;
+    float v[kVals];
+#pragma unroll
+    for (int q = 0; q < kGroups; ++q) {
+      const int off = w * kWarpElems + q * 128 + lane * 4;
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
+      if (static_cast<uint32_t>(sizeof(T)) * static_cast<uint32_t>(off + 4) <= avail) Elem<T>::four_ldg(src + off, x);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[4 * q + i] = x[i];
+    }
+    const uint32_t msk = stage_mask(v, f.t, st == 0 || st + 1 == sp.nst, sj0, L, w, lane);
+    publish(&s.red[f.par][0], msk, w, lane, false);
+    bar_filter();
+    take_stage<T, false>(s, f, &s.red[f.par][0], src, msk, base + static_cast<uint32_t>(sj0), m, tid);
+    f.par ^= 1;
+    if (f.cnt > static_cast<uint32_t>(kTrigger)) compact_any(s, f, m, tid);
+    tighten(f, m);
+  }
+  bar_filter();
+  return f;
+}
+
+// A threshold for an item with no estimate, from a sample of kSampleVals
+// values in kSampleChunks evenly spaced runs of 128 (aligned 16-byte blocks
+// inside the item): the value with as many sampled values above it as 1.5
+// times the share of m in the sample, plus 16. Returns -inf when the sample
+// gives none.
+template <class T>
+__device__ __noinline__ float sample_threshold(Smem& s, const T* row, int64_t L, int m, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(row);
+  const uintptr_t as = a & ~static_cast<uintptr_t>(15);
+  const int64_t j0 = -static_cast<int64_t>((a - as) / sizeof(T));  // item index of the aligned base
+  const int64_t span = L - j0;                                      // elements from the aligned base to the end
+#pragma unroll
+  for (int q = 0; q < kSampleRunsPerWarp; ++q) {
+    const int64_t c = w * kSampleRunsPerWarp + q;
+    const int64_t b = ((span - 128) * c / (kSampleChunks - 1)) & ~static_cast<int64_t>(3);
+    float xv[4];
+    Elem<T>::four_ldg(reinterpret_cast<const T*>(as) + b + 4 * lane, xv);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t j = j0 + b + 4 * lane + i;
+      s.fkey[c * 128 + lane * 4 + i] = (j >= 0 && j < L) ? to_key(xv[i]) : 0u;  // 0: below every key
+    }
+  }
+  bar_filter();
+  const double share = static_cast<double>(kSampleVals) * m / static_cast<double>(L);
+  const uint32_t need = min(static_cast<uint32_t>(kSampleVals - 8), static_cast<uint32_t>(1.5 * share) + 16u);
+  const uint32_t T0 = filter_kth(s, kSampleVals, need, FKey{&s}, FAll{}, tid);
+  return (T0 == 0u || T0 >= kInfKey) ? __int_as_float(0xff800000) : from_key(T0);
+}
+
+template <class T>
+__device__ __forceinline__ void load_slot(const Smem& s, int slot, int w, int lane, float (&v)[kVals]) {
+  const T* ring = reinterpret_cast<const T*>(s.ring) + slot * kStageElems;
+#pragma unroll
+  for (int q = 0; q < kGroups; ++q) {
+    float x[4];
+    Elem<T>::four(ring + w * kWarpElems + q * 128 + lane * 4, x);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[4 * q + i] = x[i];
+  }
+}
+
+// Consumer position in the ring.
+struct RingPos {
+  int slot;        // ring slot of the next stage
+  uint32_t phase;  // its full-barrier phase parity
+  uint32_t par;    // parity of the per-stage counts in s.red
+};
+
+// Streams one item (a row, or a rank's chunk of a row: L entries whose stored
+// indices are base + item index) through the ring into the candidate buffer,
+// starting from threshold f.t. Returns false when a wait gave up; the filter
+// warps then leave together.
+template <class T>
+__device__ __forceinline__ bool stream_item(Smem& s, Filter& f, RingPos& rp, const RowSpan& sp, int32_t L, uint32_t base,
+                                            int m, int tid) {
+  constexpr int kStages = stages_of<T>();
+  const int w = tid >> 5, lane = tid & 31;
+  int32_t sj0 = static_cast<int32_t>(sp.j0);  // item index of the stage's first element (< L <= INT32_MAX)
+  for (int st = 0; st < sp.nst; ++st, sj0 += kStageElems) {
+    const bool ok = mbar_wait(&s.full[rp.slot], rp.phase, &s.abort);
+    float v[kVals];
+    load_slot<T>(s, rp.slot, w, lane, v);  // values of a stage that never came are unused
+    const uint32_t msk = stage_mask(v, f.t, st == 0 || st + 1 == sp.nst, sj0, L, w, lane);
+    publish(&s.red[rp.par][0], msk, w, lane, !ok);
+    bar_filter();  // every warp's count of this stage is published
+    const T* ring = reinterpret_cast<const T*>(s.ring) + rp.slot * kStageElems;
+    if (!take_stage<T, true>(s, f, &s.red[rp.par][0], ring, msk, base + static_cast<uint32_t>(sj0), m, tid))
+      return false;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty[rp.slot]);
+    if (f.cnt > static_cast<uint32_t>(kTrigger)) compact_any(s, f, m, tid);
+    tighten(f, m);
+    rp.par ^= 1u;
+    if (++rp.slot == kStages) {
+      rp.slot = 0;
+      rp.phase ^= 1u;
+    }
+  }
+  bar_filter();  // every append is visible
+  return true;
+}
+
+template <class T>
+__device__ void filter_loop(Smem& s, const Params& p, int tid) {
+  const int lane = tid & 31;
+  const T* logits = static_cast<const T*>(p.logits);
+  const int k = p.k;
+  RingPos rp{0, 0u, 0u};
+  Filter f;
+  f.par = 0;
+  int h = 0;
+  int64_t row = blockIdx.x;
+  int32_t L_next = row < p.num_rows ? static_cast<int32_t>(clamp_len(p.lengths, row, p.row_stride)) : 0;
+  for (; row < p.num_rows; row += gridDim.x, ++h) {
+    const int32_t L = L_next;  // lengths are int32, so is every clamped length
+    if (row + gridDim.x < p.num_rows)
+      L_next = static_cast<int32_t>(clamp_len(p.lengths, row + gridDim.x, p.row_stride));
+    const int m = static_cast<int>(min64(k, L));
+    const T* rowp = logits + row * p.row_stride;
+    const RowSpan sp = row_span(rowp, L);
+    const int eb = h & 1;  // estimate written by the finisher two rows back
+    bool spec = false;
+    f.t = __int_as_float(0xff800000);
+    if (m == k) {
+      if (s.est_ok[eb] && L >= s.est_len[eb] - (s.est_len[eb] >> 3)) {
+        spec = true;
+        f.t = s.est[eb];
+      } else if (s.own_len > 0 && L >= s.own_len - (s.own_len >> 3)) {
+        spec = true;
+        f.t = s.own_key > kInfKey ? __int_as_float(0x7f800000) : from_key(s.own_key);
+      }
+    }
+    if (m == k && !spec && L >= kSampleMinLen) {
+      const float ts = sample_threshold(s, rowp, L, m, tid);
+      if (ts > __int_as_float(0xff800000)) {
+        spec = true;
+        f.t = ts;
+      }
+    }
+    if (tid == 0) s.row_t0 = f.t;  // the row's initial threshold (read by thread 0 at the row's end)
+    f.cnt = 0;
+    f.compacted = false;
+    f.strict = false;
+    f.bounded = false;
+    if (!stream_item<T>(s, f, rp, sp, L, 0u, m, tid)) return;  // a wait gave up: nothing is handed over
+    const bool reread = spec && !f.compacted && f.cnt < static_cast<uint32_t>(m);
+    if (reread) {
+      if (tid == 0) atomicOr(&g_status, kStatusReread);
+      f = refilter_from_global<T>(s, f, sp, L, 0u, m, tid);
+    }
+    if (f.cnt > static_cast<uint32_t>(kHandCap)) compact_any(s, f, m, tid);
+    if (tid == 0 && m == k) {
+      // carried to the CTA's next row: a speculative threshold that passed at
+      // least m values of this row (it needed no re-read), else the bound the
+      // filter ended with. A compaction's cut is a poor carry: it can sit
+      // just under this row's m-th value and above a similar row's.
+      if (spec && !reread) {
+        s.own_key = to_key(s.row_t0);
+        s.own_len = L;
+      } else if (f.bounded) {
+        s.own_key = f.last_key;
+        s.own_len = L;
+      }
+    }
+    bar_filter();  // the own estimate is read at the next row's start
+    // hand over: wait until the finishers released the previous handover
+    const bool ok = mbar_wait_sleep(&s.hempty, (h & 1) ^ 1, &s.abort);
+    if (bar_filter_any(!ok)) return;
+    for (int e = tid; e < static_cast<int>(f.cnt); e += kFilterThreads) {
+      s.hkey[e] = s.fkey[e];
+      s.hidx[e] = s.fidx[e];
+    }
+    if (tid == 0) {
+      s.h_row = row;
+      s.h_len = L;
+      s.h_n = static_cast<int32_t>(f.cnt);
+      s.h_m = m;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.hfull);
+  }
+}
+
+// ---------------------------------------------------------- finisher
+// Ranks candidates hkey/hidx [0, n) by the composite C = (kmax - key) << 32 |
+// index (ascending C = key descending, index ascending; all C distinct) and
+// writes the first m to the output row. Buckets are 12-bit slices of C: count,
+// scan, then find the bucket holding rank m-1. While a bucket at or before it
+// is large, the range shrinks to the buckets up to it (everything after has
+// rank >= m) and the count repeats. Then the candidates are grouped by bucket
+// and each one's rank is its bucket's start plus the number of bucket members
+// ahead of it. In set mode (DSA_FLAG_UNSORTED) only the bucket holding rank
+// m-1 is ranked; the rest of the top m is written in bucket order.
+// NT threads (192: the finisher warps; 256: the filter warps of a cluster's
+// leader) synchronise on named barrier BAR.
+template <int NT, int BAR>
+struct Finisher {
+  static constexpr int kWarps = NT / 32;
+  static constexpr int kBuckets = NT == 192 ? 3840 : 4096;
+  static constexpr int kScanPer = kBuckets / NT;  // counters per thread
+  static_assert(kBuckets <= kBucketMax && kBuckets >= 2048 && kScanPer % 4 == 0 && kWarps <= kFilterWarps,
+                "bucket counters split evenly over the threads; bucket_shift narrows a slice by one bit at most");
+
+  __device__ __forceinline__ static void bar() { asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory"); }
+
+  __device__ __forceinline__ static int bucket_shift(uint64_t cmax) {
+    const int bits = cmax ? 64 - __clzll(static_cast<long long>(cmax)) : 0;
+    int sh = bits > 12 ? bits - 12 : 0;  // cmax >> sh < 4096
+    if ((cmax >> sh) >= static_cast<uint64_t>(kBuckets)) ++sh;
+    return sh;
+  }
+
+  // index -> output value: the optional table maps a row-local index to the
+  // caller's value (-1 passes through)
+  __device__ __forceinline__ static int32_t emit(const Params& p, int64_t row, int32_t idx) {
+    if (p.table == nullptr || idx < 0) return idx;
+    return __ldg(p.table + row * p.table_stride + idx);
+  }
+
+  // Candidates [0, n) ordered in place by (key descending, index ascending)
+  // with a bitonic network over the next power of two (padding keys 0 sort
+  // last), then the first m written. Ends with a barrier.
+  __device__ __noinline__ static void finish_sorted(Smem& s, int n, int m, int k, int64_t row, const Params& p,
+                                                    int fid) {
+    int32_t* o = p.out + row * static_cast<int64_t>(k);
+    int N = 1;
+    while (N < n) N <<= 1;
+    for (int e = n + fid; e < N; e += NT) {
+      s.hkey[e] = 0u;
+      s.hidx[e] = 0xFFFFFFFFu;
+    }
+    bar();
+    for (int size = 2; size <= N; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int t = fid; t < (N >> 1); t += NT) {
+          const int i = 2 * t - (t & (stride - 1));
+          const int j = i + stride;
+          const uint32_t ki = s.hkey[i], ii = s.hidx[i], kj = s.hkey[j], ij = s.hidx[j];
+          const bool j_first = kj > ki || (kj == ki && ij < ii);  // j belongs before i
+          if (j_first == ((i & size) == 0)) {
+            s.hkey[i] = kj;
+            s.hidx[i] = ij;
+            s.hkey[j] = ki;
+            s.hidx[j] = ii;
+          }
+        }
+        bar();
+      }
+    }
+    const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
+    for (int q = fid; q < m; q += NT) {
+      o[q] = emit(p, row, static_cast<int32_t>(s.hidx[q]));
+      if (q == k - 1) s.rec[0] = s.hkey[q];
+      if (q == a) s.rec[1] = s.hkey[q];
+    }
+    bar();
+  }
+
+  // Ranks n candidates and writes the row: m indices, then -1 up to k.
+  __device__ __noinline__ static void finish(Smem& s, int n, int m, int k, int64_t row, const Params& p, int fid) {
+    const int fw = fid >> 5, lane = fid & 31;
+    int32_t* o = p.out + row * static_cast<int64_t>(k);
+    for (int q = m + fid; q < k; q += NT) o[q] = -1;
+    if (n <= 0) return;
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, imax = 0u;
+    for (int e = fid; e < n; e += NT) {
+      const uint32_t key = s.hkey[e];
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
+      imax = max(imax, s.hidx[e]);
+    }
+    kmin = __reduce_min_sync(kFull, kmin);
+    kmax = __reduce_max_sync(kFull, kmax);
+    imax = __reduce_max_sync(kFull, imax);
+    if (lane == 0) {
+      s.nred[0][fw] = kmin;
+      s.nred[1][fw] = kmax;
+      s.nred[2][fw] = imax;
+    }
+    bar();
+#pragma unroll
+    for (int ww = 0; ww < kWarps; ++ww) {
+      kmin = min(kmin, s.nred[0][ww]);
+      kmax = max(kmax, s.nred[1][ww]);
+      imax = max(imax, s.nred[2][ww]);
+    }
+    uint64_t cmax = (static_cast<uint64_t>(kmax - kmin) << 32) | imax;
+    int sh = bucket_shift(cmax);
+    auto comp = [&](uint32_t key, uint32_t idx) -> uint64_t {
+      return (static_cast<uint64_t>(kmax - key) << 32) | idx;
+    };
+    uint4* bc4 = reinterpret_cast<uint4*>(&s.bcnt[fid * kScanPer]);
+    const uint32_t mm1 = static_cast<uint32_t>(m - 1);
+    uint32_t big = 0;
+    for (int pass = 0;; ++pass) {
+#pragma unroll
+      for (int i = 0; i < kScanPer / 4; ++i) bc4[i] = make_uint4(0u, 0u, 0u, 0u);
+      bar();
+      for (int e = fid; e < n; e += NT) {
+        const uint64_t c = comp(s.hkey[e], s.hidx[e]);
+        if (c <= cmax) atomicAdd(&s.bcnt[static_cast<uint32_t>(c >> sh)], 1u);
+      }
+      bar();
+      // exclusive scan: thread fid owns counters [kScanPer fid, kScanPer (fid + 1))
+      uint32_t c[kScanPer], sum = 0;
+#pragma unroll
+      for (int i = 0; i < kScanPer / 4; ++i) {
+        const uint4 q = bc4[i];
+        c[4 * i + 0] = q.x;
+        c[4 * i + 1] = q.y;
+        c[4 * i + 2] = q.z;
+        c[4 * i + 3] = q.w;
+        sum += q.x + q.y + q.z + q.w;
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t t = __shfl_up_sync(kFull, incl, d);
+        if (lane >= d) incl += t;
+      }
+      if (lane == 31) s.nred[3][fw] = incl;
+      bar();
+      uint32_t run = incl - sum;
+      for (int ww = 0; ww < fw; ++ww) run += s.nred[3][ww];
+      const uint32_t run0 = run;
+#pragma unroll
+      for (int i = 0; i < kScanPer / 4; ++i) {
+        uint4 q;
+        q.x = run;
+        run += c[4 * i + 0];
+        q.y = run;
+        run += c[4 * i + 1];
+        q.z = run;
+        run += c[4 * i + 2];
+        q.w = run;
+        run += c[4 * i + 3];
+        bc4[i] = q;
+      }
+      // the bucket holding rank m-1 (exactly one thread finds it)
+      run = run0;
+#pragma unroll
+      for (int i = 0; i < kScanPer; ++i) {
+        if (run <= mm1 && mm1 < run + c[i]) s.bc[4] = static_cast<uint32_t>(fid * kScanPer + i);
+        run += c[i];
+      }
+      bar();
+      const uint32_t bm = s.bc[4];
+      big = 0;  // largest bucket at or before bm
+#pragma unroll
+      for (int i = 0; i < kScanPer; ++i)
+        if (static_cast<uint32_t>(fid * kScanPer + i) <= bm) big = max(big, c[i]);
+      big = __reduce_max_sync(kFull, big);
+      if (lane == 0) s.nred[4][fw] = big;
+      bar();
+#pragma unroll
+      for (int ww = 0; ww < kWarps; ++ww) big = max(big, s.nred[4][ww]);
+      if (big <= static_cast<uint32_t>(kSmallBucket) || sh == 0 || pass == kSortPasses - 1) break;
+      cmax = ((static_cast<uint64_t>(bm) + 1u) << sh) - 1u;
+      sh = bucket_shift(cmax);
+      bar();  // bc[4] and nred[4] are rewritten by the next pass
+    }
+    if (big > static_cast<uint32_t>(kBigBucket)) {
+      // many candidates share a bucket (values on a coarse grid): counting
+      // ranks inside it would be quadratic, so sort everything instead
+      finish_sorted(s, n, m, k, row, p, fid);
+      return;
+    }
+    for (int e = fid; e < n; e += NT) {
+      const uint64_t cc = comp(s.hkey[e], s.hidx[e]);
+      if (cc > cmax) continue;
+      const uint32_t q = atomicAdd(&s.bcnt[static_cast<uint32_t>(cc >> sh)], 1u);
+      s.perm[q] = static_cast<uint16_t>(e);
+    }
+    bar();  // bcnt[b] is now the end of bucket b (= start of b + 1)
+    const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
+    if (p.flags & kUnsorted) {
+      // set mode: positions before the bucket holding rank m-1 are taken as
+      // they lie (bucket order); only that bucket's members are ranked
+      const uint32_t bm = s.bc[4];
+      const uint32_t s0 = bm ? s.bcnt[bm - 1] : 0u, s1 = s.bcnt[bm];
+      for (uint32_t q = fid; q < s0; q += NT) {
+        const uint32_t e = s.perm[q];
+        s.ostage[q] = static_cast<int32_t>(s.hidx[e]);
+        if (q == static_cast<uint32_t>(a)) s.rec[1] = s.hkey[e];
+      }
+      for (uint32_t q = s0 + fid; q < s1; q += NT) {
+        const uint32_t e = s.perm[q];
+        const uint32_t key = s.hkey[e], idx = s.hidx[e];
+        uint32_t r = s0;
+        for (uint32_t q2 = s0; q2 < s1; ++q2) {
+          const uint32_t j = s.perm[q2];
+          const uint32_t kj = s.hkey[j], ij = s.hidx[j];
+          r += kj > key || (kj == key && ij < idx);
+        }
+        if (r < static_cast<uint32_t>(m)) {
+          s.ostage[r] = static_cast<int32_t>(idx);
+          if (r == static_cast<uint32_t>(k - 1)) s.rec[0] = key;
+          if (r == static_cast<uint32_t>(a)) s.rec[1] = key;
+        }
+      }
+    } else {
+      for (int e = fid; e < n; e += NT) {
+        const uint32_t key = s.hkey[e], idx = s.hidx[e];
+        const uint64_t cc = comp(key, idx);
+        if (cc > cmax) continue;
+        const uint32_t b = static_cast<uint32_t>(cc >> sh);
+        const uint32_t s0 = b ? s.bcnt[b - 1] : 0u, s1 = s.bcnt[b];
+        if (s0 >= static_cast<uint32_t>(m)) continue;
+        uint32_t r = s0;
+        for (uint32_t q = s0; q < s1; ++q) {
+          const uint32_t j = s.perm[q];
+          const uint32_t kj = s.hkey[j], ij = s.hidx[j];
+          r += kj > key || (kj == key && ij < idx);
+        }
+        if (r < static_cast<uint32_t>(m)) {
+          s.ostage[r] = static_cast<int32_t>(idx);
+          if (r == static_cast<uint32_t>(k - 1)) s.rec[0] = key;
+          if (r == static_cast<uint32_t>(a)) s.rec[1] = key;
+        }
+      }
+    }
+    bar();
+    for (int q = fid; q < m; q += NT) o[q] = emit(p, row, s.ostage[q]);
+  }
+};
+
+using RowFinisher = Finisher<kFinishThreads, 2>;
+using LeaderFinisher = Finisher<kFilterThreads, 1>;
+
+__device__ void finish_loop(Smem& s, const Params& p, int fid) {
+  const int lane = fid & 31;
+  const int k = p.k;
+  int h = 0;
+  for (int64_t row = blockIdx.x; row < p.num_rows; row += gridDim.x, ++h) {
+    const bool ok = mbar_wait_sleep(&s.hfull, h & 1, &s.abort);
+    if (bar_any<2, kFinishThreads>(!ok)) return;  // the filter warps left: nothing more comes
+    const int n = s.h_n, m = s.h_m;
+    const int64_t L = s.h_len;
+    RowFinisher::finish(s, n, m, k, s.h_row, p, fid);
+    if (fid == 0) {
+      bool est_ok = false;
+      float e = 0.f;
+      if (n > 0 && m == k) {
+        const uint32_t kt = s.rec[0], ka = s.rec[1];
+        const float vt = from_key(kt), va = from_key(ka);
+        e = vt - 0.5f * (va - vt);
+        est_ok = kt != kNanKey && ka != kNanKey && isfinite(e);
+      }
+      s.est[h & 1] = e;
+      s.est_len[h & 1] = L;
+      s.est_ok[h & 1] = est_ok ? 1 : 0;
+    }
+    RowFinisher::bar();  // every read of the handover is done, the estimate written
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.hempty);
+  }
+}
+
+// ---------------------------------------------------------- producer
+// Issues one item's stages into the ring. Returns false when a wait gave up.
+template <class T>
+__device__ __forceinline__ bool produce_span(Smem& s, const RowSpan& sp, int& slot, uint32_t& phase, long long& gi,
+                                             long long skip, uint32_t& armed, uint32_t& arm_par) {
+  constexpr int kStages = stages_of<T>();
+  constexpr uint32_t kStageBytes = kStageElems * sizeof(T);
+  for (int st = 0; st < sp.nst; ++st, ++gi) {
+    if (!mbar_wait_sleep(&s.empty[slot], phase ^ 1u, &s.abort)) return false;
+    if (gi != skip) {
+      const uint32_t bytes = st + 1 == sp.nst ? sp.last_bytes : kStageBytes;
+      fence_proxy_async();
+      mbar_arrive_expect_tx(&s.full[slot], bytes);
+      bulk_g2s(s.ring + static_cast<uint32_t>(slot) * kStageBytes, sp.src + static_cast<uint64_t>(st) * kStageBytes,
+               bytes, &s.full[slot]);
+      armed |= 1u << slot;
+      arm_par = (arm_par & ~(1u << slot)) | (phase << slot);
+    }
+    if (++slot == kStages) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+  return true;
+}
+
+// Before returning, on the normal path and after an abort alike, the producer
+// waits until the last copy it issued into each slot has landed, so the CTA
+// never exits with a bulk copy still writing into its shared memory.
+__device__ __forceinline__ void producer_drain(Smem& s, uint32_t armed, uint32_t arm_par) {
+  for (int i = 0; i < kMaxStages; ++i)
+    if ((armed >> i) & 1u) mbar_drain(&s.full[i], (arm_par >> i) & 1u);
+}
+
+template <class T>
+__device__ void produce_loop(Smem& s, const Params& p) {
+  const T* logits = static_cast<const T*>(p.logits);
+  int slot = 0;
+  uint32_t phase = 0u, armed = 0u, arm_par = 0u;
+  const long long skip = g_skip_stage;  // test hook: a stage left unissued
+  long long gi = 0;                     // stages this CTA has passed (issued or skipped)
+  for (int64_t row = blockIdx.x; row < p.num_rows; row += gridDim.x) {
+    const int64_t L = clamp_len(p.lengths, row, p.row_stride);
+    if (!produce_span<T>(s, row_span(logits + row * p.row_stride, L), slot, phase, gi, skip, armed, arm_par)) break;
+  }
+  producer_drain(s, armed, arm_par);
+}
+
+// ---------------------------------------------------------- cluster mode
+// After streaming, rank `rank` holds n_r candidates in fkey/fidx, a superset
+// of its chunk's top min(m, chunk) (none if a wait gave up). The filter warps
+// of every rank run the merge; at the leader (rank 0) the survivors end in
+// hkey/hidx. Returns the number gathered there. The producer warp mirrors
+// every cluster barrier (s.final_bar tells it how many there are).
+__device__ __noinline__ uint32_t cluster_merge(Smem& s, uint32_t n_r, uint32_t m, bool aborted, uint32_t rank,
+                                               uint32_t ncta, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  uint32_t nbar = 0;
+  uint32_t* phist = s.bcnt;        // [2][256], per rank, read by the others
+  uint32_t* ghist = s.bcnt + 512;  // [256], cluster sums
+  // ---- phase 1: publish (count, min key, max key, gave up) of this rank
+  uint32_t mn, mx;
+  filter_minmax(s, static_cast<int>(n_r), FKey{&s}, FAll{}, mn, mx, tid);
+  if (tid == 0) {
+    s.pub[0] = n_r;
+    s.pub[1] = mn;
+    s.pub[2] = mx;
+    s.pub[3] = aborted ? 1u : 0u;
+  }
+  cluster_barrier();
+  ++nbar;
+  if (w == 0) {
+    uint32_t n = 0, lo_r = 0xFFFFFFFFu, hi_r = 0u, ab = 0u;
+    if (lane < static_cast<int>(ncta)) {
+      const uint32_t a = dsmem_map(smem_addr(&s.pub[0]), lane);
+      n = dsmem_ld(a);
+      lo_r = dsmem_ld(a + 4);
+      hi_r = dsmem_ld(a + 8);
+      ab = dsmem_ld(a + 12);
+    }
+    const bool full_rank = lane < static_cast<int>(ncta) && n >= m;
+    const uint32_t N = __reduce_add_sync(kFull, n);
+    const uint32_t gmin = __reduce_min_sync(kFull, lo_r);
+    const uint32_t gmax = __reduce_max_sync(kFull, hi_r);
+    // a rank holding at least m entries at or above its min bounds the m-th key from below
+    const uint32_t B = __reduce_max_sync(kFull, full_rank ? lo_r : 0u);
+    const bool any_full = __ballot_sync(kFull, full_rank) != 0;
+    const bool any_ab = __ballot_sync(kFull, ab != 0u) != 0;
+    if (lane == 0) {
+      s.bc[2] = N;
+      s.bc[3] = any_full ? B : gmin;
+      s.bc[4] = gmax;
+      s.bc[5] = gmin;
+      s.abort_any = any_ab ? 1u : 0u;
+    }
+  }
+  bar_filter();
+  const uint32_t N = s.bc[2];
+  uint32_t lo = s.bc[3], hi = s.bc[4];
+  const uint32_t gmin = s.bc[5];
+  bar_filter();
+  uint32_t need = m;
+  bool exact = false;
+  if (N <= static_cast<uint32_t>(kHandCap)) {
+    lo = gmin;  // everything fits at the leader
+  } else {
+    // ---- phase 2: cluster-wide histogram rounds until the survivors fit
+    int hp = 0;
+    for (int round = 0;; ++round) {
+      if (lo == hi || round == kRounds + 1) {
+        if (lo != hi && tid == 0) atomicOr(&g_status, kStatusSelectBroken);
+        exact = true;
+        break;
+      }
+      const int sh = window_shift(lo, hi);
+      uint32_t* ph = phist + 256 * hp;
+      ph[tid] = 0u;  // kFilterThreads == 256
+      if (tid == 0) s.bc[0] = 0xFFFFFFFFu;
+      bar_filter();
+      digit_histogram(ph, static_cast<int>(n_r), FKey{&s}, FAll{}, lo, hi, sh, tid);
+      cluster_barrier();
+      ++nbar;
+      {
+        const uint32_t a = smem_addr(&ph[tid]);
+        uint32_t g = 0;
+        for (uint32_t r = 0; r < ncta; ++r) g += dsmem_ld(dsmem_map(a, r));
+        ghist[tid] = g;
+      }
+      bar_filter();
+      if (w == 0) find_bucket_warp0(ghist, need, s.bc, lane);
+      bar_filter();
+      if (s.bc[0] == 0xFFFFFFFFu) {  // identical on every rank: the same sums
+        if (tid == 0) atomicOr(&g_status, kStatusSelectBroken);
+        exact = true;
+        lo = hi;
+        bar_filter();
+        break;
+      }
+      const uint32_t b = s.bc[0], above_b = s.bc[1];
+      need -= above_b;
+      const uint32_t S = (m - need) + ghist[b];  // keys above the bucket + keys in it
+      narrow(lo, hi, sh, b);
+      bar_filter();
+      hp ^= 1;
+      if (S <= static_cast<uint32_t>(kHandCap)) break;
+    }
+  }
+  if (tid == 0) s.final_bar = nbar + 2;  // phases 3 and 4 end with one cluster barrier each
+  // ---- phase 3: publish this rank's survivor counts
+  // exact: keep key > T plus a rank-ordered share of key == T; else keep key >= lo
+  const uint32_t T = exact ? lo : lo - 1u;
+  uint32_t g_r, q_r;
+  count_gt_eq(s, static_cast<int>(n_r), T, g_r, q_r, tid);
+  if (tid == 0) {
+    s.pub[4] = g_r;
+    s.pub[5] = exact ? q_r : 0u;
+  }
+  cluster_barrier();
+  ++nbar;
+  if (w == 0) {
+    uint32_t g = 0, q = 0;
+    if (lane < static_cast<int>(ncta)) {
+      const uint32_t a = dsmem_map(smem_addr(&s.pub[4]), lane);
+      g = dsmem_ld(a);
+      q = dsmem_ld(a + 4);
+    }
+    // ranks hold contiguous, increasing index ranges: rank order is index order
+    uint32_t q_incl = q;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(kFull, q_incl, o);
+      if (lane >= o) q_incl += v;
+    }
+    const uint32_t q_excl = q_incl - q;
+    const uint32_t keep_q = exact ? (need > q_excl ? min(q, need - q_excl) : 0u) : 0u;
+    const uint32_t cnt = g + keep_q;
+    uint32_t c_incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(kFull, c_incl, o);
+      if (lane >= o) c_incl += v;
+    }
+    if (lane == static_cast<int>(rank)) {
+      s.bc[6] = c_incl - cnt;  // my offset at the leader
+      s.bc[7] = keep_q;
+    }
+    const uint32_t total = __shfl_sync(kFull, c_incl, 31);
+    if (lane == 0) s.bc[2] = total;
+  }
+  bar_filter();
+  const uint32_t my_off = s.bc[6], my_keep = s.bc[7], total = s.bc[2];
+  bar_filter();
+  // ---- phase 4: copy survivors into the leader at rank-ordered offsets
+  const uint32_t rkey = dsmem_map(smem_addr(&s.hkey[0]), 0);
+  const uint32_t ridx = dsmem_map(smem_addr(&s.hidx[0]), 0);
+  if (exact && my_keep > 0u) {
+    // this rank's share of the tied key: its my_keep lowest indices
+    const uint32_t I = my_keep < q_r ? tie_cut(s, static_cast<int>(n_r), T, my_keep, tid) : 0xFFFFFFFFu;
+    keep_pass<true, true>(s, static_cast<int>(n_r), T, I, tid, rkey, ridx, my_off);
+  } else {
+    keep_pass<false, true>(s, static_cast<int>(n_r), T, 0u, tid, rkey, ridx, my_off);
+  }
+  cluster_barrier();
+  ++nbar;
+  return total;
+}
+
+template <class T>
+__device__ __noinline__ void cluster_row(Smem& s, const Params& p, int tid) {
+  const int w = tid >> 5, lane = tid & 31;  // warp kClusterWarp is the producer
+  const uint32_t rank = cluster_rank(), ncta = cluster_size();
+  const int64_t row = cluster_index();
+  const T* rowp = static_cast<const T*>(p.logits) + row * p.row_stride;
+  const int64_t L = clamp_len(p.lengths, row, p.row_stride);
+  const int k = p.k;
+  const uint32_t m = static_cast<uint32_t>(min64(k, L));
+  if (m == 0) {  // the same for every CTA of the cluster: no merge, no barrier
+    if (rank == 0 && w < kFilterWarps)
+      for (int q = tid; q < k; q += kFilterThreads) p.out[row * static_cast<int64_t>(k) + q] = -1;
+    return;
+  }
+  int64_t chunk = (L + ncta - 1) / ncta;
+  chunk = (chunk + 7) & ~static_cast<int64_t>(7);
+  const int64_t c0 = min64(L, static_cast<int64_t>(rank) * chunk);
+  const int64_t c1 = min64(L, c0 + chunk);
+  const int32_t Lc = static_cast<int32_t>(c1 - c0);
+  const RowSpan sp = row_span(rowp + c0, Lc);
+  if (w == kClusterWarp) {
+    // producer: lane 0 streams the chunk; then the whole warp mirrors the
+    // merge's cluster barriers, leaving after the last one
+    if (lane == 0) {
+      int slot = 0;
+      uint32_t phase = 0u, armed = 0u, arm_par = 0u;
+      long long gi = 0;
+      produce_span<T>(s, sp, slot, phase, gi, g_skip_stage, armed, arm_par);
+      producer_drain(s, armed, arm_par);
+    }
+    __syncwarp();
+    for (uint32_t i = 1;; ++i) {
+      cluster_barrier();
+      const volatile uint32_t* fb = &s.final_bar;
+      if (*fb == i) break;
+    }
+    return;
+  }
+  // filter warps: this rank's chunk, then the merge
+  const uint32_t m_r = min(m, static_cast<uint32_t>(Lc));
+  Filter f;
+  f.par = 0;
+  f.t = __int_as_float(0xff800000);
+  bool spec = false;
+  if (Lc >= kSampleMinLen && m_r > 0) {
+    const float ts = sample_threshold(s, rowp + c0, Lc, static_cast<int>(m_r), tid);
+    if (ts > __int_as_float(0xff800000)) {
+      spec = true;
+      f.t = ts;
+    }
+  }
+  f.cnt = 0;
+  f.compacted = false;
+  f.strict = false;
+  f.bounded = false;
+  RingPos rp{0, 0u, 0u};
+  const bool ok = stream_item<T>(s, f, rp, sp, Lc, static_cast<uint32_t>(c0), static_cast<int>(m_r), tid);
+  if (!ok) {
+    f.cnt = 0;  // no candidates from this rank; it still takes part in the merge
+  } else {
+    if (spec && !f.compacted && f.cnt < m_r) {
+      if (tid == 0) atomicOr(&g_status, kStatusReread);
+      f = refilter_from_global<T>(s, f, sp, Lc, static_cast<uint32_t>(c0), static_cast<int>(m_r), tid);
+    }
+    if (f.cnt > static_cast<uint32_t>(kHandCap)) compact_any(s, f, static_cast<int>(m_r), tid);
+  }
+  const uint32_t total = cluster_merge(s, f.cnt, m, !ok, rank, ncta, tid);
+  if (rank != 0) return;
+  if (s.abort_any) {  // some rank gave up: no valid result for this row
+    for (int q = tid; q < k; q += kFilterThreads) p.out[row * static_cast<int64_t>(k) + q] = -1;
+    return;
+  }
+  LeaderFinisher::finish(s, static_cast<int>(total), static_cast<int>(m), k, row, p, tid);
+}
+
+}  // namespace rows
+
+// Many rows (cluster size 1): grid = min(num_rows, SMs), one CTA per SM,
+// rows strided by the grid, 480 threads. A cluster per row: grid = num_rows *
+// cluster size, 288 threads.
+template <class T>
+__global__ void __launch_bounds__(rows::kThreads, 1) topk_kernel(const rows::Params p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  rows::Smem& s = *reinterpret_cast<rows::Smem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool clustered = cluster_size() > 1;
+  if (tid == 0) {
+    for (int i = 0; i < rows::kMaxStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], rows::kFilterWarps);
+    }
+    mbar_init(&s.hfull, rows::kFilterWarps);
+    mbar_init(&s.hempty, rows::kFinishWarps);
+    for (int i = 0; i < 2; ++i) {
+      s.est_ok[i] = 0;
+      s.est[i] = 0.f;
+      s.est_len[i] = 0;
+    }
+    s.own_key = 0u;
+    s.own_len = 0;
+    s.abort = 0u;
+    s.abort_any = 0u;
+    s.final_bar = 0u;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_enter();  // every thread: inputs and outputs are touched only after this
+  if (clustered) {
+    rows::cluster_row<T>(s, p, tid);
+  } else if (warp < rows::kFilterWarps) {
+    rows::filter_loop<T>(s, p, tid);
+  } else if (warp < rows::kProducerWarp) {
+    rows::finish_loop(s, p, tid - rows::kFilterThreads);
+  } else if (lane == 0) {
+    rows::produce_loop<T>(s, p);
+  }
+}
+
+}  // namespace dsa

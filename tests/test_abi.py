@@ -31,8 +31,8 @@ def pkg():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("dsa_topk", "dsa_topk_host", "dsa_topk_plan", "dsa_topk_device_status",
-              "dsa_topk_strerror", "dsa_topk_version"):
+    for n in ("dsa_topk", "dsa_topk_ex", "dsa_topk_host", "dsa_topk_plan", "dsa_topk_device_status",
+              "dsa_topk_set_test_hooks", "dsa_topk_strerror", "dsa_topk_version"):
         assert n in names
 
 
@@ -50,7 +50,7 @@ def test_library_exports_every_declared_symbol(pkg):
 def test_strerror_and_version(pkg):
     assert pkg.version() >= 100
     assert pkg.strerror(0) == "success"
-    for code in range(-9, 0):
+    for code in range(-11, 0):
         assert pkg.strerror(code) and pkg.strerror(code) != pkg.strerror(1)
 
 
@@ -81,3 +81,22 @@ def test_plan_rejects_bad_sizes(pkg):
     assert pkg.lib.dsa_topk_plan(4, 16, 0, None, None) == -2
     assert pkg.lib.dsa_topk_plan(4, 0, 8, None, None) == -3
     assert pkg.lib.dsa_topk_plan(-4, 16, 8, None, None) == -4
+
+
+@pytest.mark.parametrize("args,code", [
+    # (logits, dtype, row_stride, lengths, num_rows, k, flags, table, table_stride, out)
+    ((8, 3, 16, 8, 2, 4, 0, 0, 0, 8), -10),    # unknown dtype
+    ((8, 0, 16, 8, 2, 4, 2, 0, 0, 8), -11),    # unknown flag bit
+    ((8, 0, 16, 8, 2, 4, 0, 8, 0, 8), -3),     # table without a positive stride
+    ((10, 1, 16, 8, 2, 4, 0, 0, 0, 8), 0),     # bf16 needs 2-byte alignment only: reaches the device check
+    ((9, 1, 16, 8, 2, 4, 0, 0, 0, 8), -6),     # misaligned bf16 logits
+    ((8, 0, 16, 8, 2, 4, 0, 10, 3, 8), -6),    # misaligned table
+    ((8, 2, 16, 8, 0, 4, 1, 0, 0, 8), 0),      # zero rows: no-op
+])
+def test_ex_argument_errors(pkg, args, code):
+    lo, dt, stride, le, rows, k, flags, tab, ts, out = args
+    rc = pkg.lib.dsa_topk_ex(lo or None, dt, stride, le or None, rows, k, flags, tab or None, ts, out or None, None)
+    if code == 0 and rows:
+        assert rc in (0, -7)  # -7: no sm_100a device here
+    else:
+        assert rc == code
