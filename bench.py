@@ -246,9 +246,11 @@ def _time_workload(dsa, torch, peak, wl, dtype=None, unsorted=False, table=False
     kw = {"unsorted": unsorted, "index_table": tab}
     n_calls = max(R, min(256, max(8, int(2e9 // max(vb, 1)))))
     cold = [(lambda c=copies[i % R]: dsa.dsa_topk(c, lengths, wl.k, out=out, **kw)) for i in range(n_calls)]
+    dsa.device_status(clear=True)
     us_cold = time_graph(dsa, torch, cold)
     warm = [(lambda: dsa.dsa_topk(base, lengths, wl.k, out=out, **kw)) for _ in range(min(n_calls, 64))]
     us_warm = time_graph(dsa, torch, warm)
+    status = dsa.device_status(clear=True)
     cs, grid = dsa.plan(wl.num_rows, wl.row_stride, wl.k)
     gbs = vb / us_cold / 1e3
     res = {
@@ -256,6 +258,7 @@ def _time_workload(dsa, torch, peak, wl, dtype=None, unsorted=False, table=False
         "valid_gbs": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
         "us_per_call_warm_l2": round(us_warm, 3), "valid_bytes": vb,
         "rotating_copies": R, "cluster_size": cs, "grid": grid,
+        "device_status": status,  # bit 2: some row was re-read after a speculative threshold (info)
     }
     del copies, base, out, tab
     torch.cuda.empty_cache()

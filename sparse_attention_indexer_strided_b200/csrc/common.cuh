@@ -70,19 +70,28 @@ __device__ __forceinline__ unsigned long long global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Bounded wait. Returns false after g_wait_limit_ns (recording the status bit
-// and raising the CTA's abort flag), or at once when another thread of the CTA
-// has raised that flag: the first wait that gives up ends every later one.
-__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity, volatile uint32_t* abort) {
+// Per-CTA wait control in shared memory: the abort flag raised by the first
+// wait that gives up, and the time limit of every wait (copied from
+// g_wait_limit_ns once at kernel start, so that a wait's slow path never
+// stalls on a global load before it looks at its barrier again).
+struct WaitCtl {
+  uint32_t abort;
+  uint32_t pad;
+  unsigned long long limit_ns;
+};
+
+// Bounded wait. Returns false after the limit (recording the status bit and
+// raising the CTA's abort flag), or at once when another thread of the CTA has
+// raised that flag: the first wait that gives up ends every later one.
+__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity, WaitCtl* ctl) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
-  const unsigned long long lim = g_wait_limit_ns;
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (global_ns() - t0 > lim) {
+    if (*reinterpret_cast<volatile uint32_t*>(&ctl->abort)) return false;
+    if (global_ns() - t0 > ctl->limit_ns) {
       atomicOr(&g_status, kStatusWaitTimeout);
-      *abort = 1u;
+      *reinterpret_cast<volatile uint32_t*>(&ctl->abort) = 1u;
       return false;
     }
   }
@@ -102,16 +111,15 @@ __device__ __forceinline__ bool mbar_try_wait_hint(unsigned long long* bar, uint
 }
 // Bounded wait for waits that are often long (a role idling until another
 // catches up): sleeps in the barrier instead of spinning.
-__device__ __forceinline__ bool mbar_wait_sleep(unsigned long long* bar, uint32_t parity, volatile uint32_t* abort) {
+__device__ __forceinline__ bool mbar_wait_sleep(unsigned long long* bar, uint32_t parity, WaitCtl* ctl) {
   if (mbar_try_wait_hint(bar, parity, 2000u)) return true;
   const unsigned long long t0 = global_ns();
-  const unsigned long long lim = g_wait_limit_ns;
   for (;;) {
     if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
-    if (*abort) return false;
-    if (global_ns() - t0 > lim) {
+    if (*reinterpret_cast<volatile uint32_t*>(&ctl->abort)) return false;
+    if (global_ns() - t0 > ctl->limit_ns) {
       atomicOr(&g_status, kStatusWaitTimeout);
-      *abort = 1u;
+      *reinterpret_cast<volatile uint32_t*>(&ctl->abort) = 1u;
       return false;
     }
   }
@@ -119,12 +127,11 @@ __device__ __forceinline__ bool mbar_wait_sleep(unsigned long long* bar, uint32_
 // Drain: waits (bounded, ignoring the abort flag) until an issued bulk copy
 // has landed, so that no copy is still writing into shared memory when the
 // CTA exits. Copies from valid global memory always complete.
-__device__ __forceinline__ void mbar_drain(unsigned long long* bar, uint32_t parity) {
+__device__ __forceinline__ void mbar_drain(unsigned long long* bar, uint32_t parity, const WaitCtl* ctl) {
   if (mbar_try_wait(bar, parity)) return;
   const unsigned long long t0 = global_ns();
-  const unsigned long long lim = g_wait_limit_ns;
   while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > lim) {
+    if (global_ns() - t0 > ctl->limit_ns) {
       atomicOr(&g_status, kStatusWaitTimeout);
       return;
     }

@@ -33,8 +33,8 @@
 // m values pass it, the filter warps re-read the row from global memory with
 // no threshold; the result is exact either way, only the time changes.
 //
-// Cluster mode (a cluster of C CTAs per row, 288 threads: filter warps and a
-// producer warp, no finisher warps): rank r streams the contiguous chunk r of
+// Cluster mode (a cluster of C CTAs per row, 384 threads: filter warps and a
+// producer warpgroup, no finisher warps): rank r streams the contiguous chunk r of
 // the row exactly as a row is streamed above, keeping a superset of the
 // chunk's top min(m, chunk). The ranks then merge through distributed shared
 // memory (SGLang PR #34167 code excerpt, TopKCluster::forward: per-rank
@@ -64,9 +64,21 @@ constexpr int kFilterThreads = kFilterWarps * 32;  // 256
 constexpr int kFinishWarps = 6;
 constexpr int kFinishThreads = kFinishWarps * 32;  // 192
 constexpr int kProducerWarp = kFilterWarps + kFinishWarps;
-constexpr int kThreads = (kProducerWarp + 1) * 32;      // 480: many-row mode
+constexpr int kThreads = 16 * 32;                       // 512: many-row mode (4 warpgroups; warp 15 idle)
 constexpr int kClusterWarp = kFilterWarps;              // cluster mode: the producer warp
-constexpr int kClusterThreads = (kFilterWarps + 1) * 32;  // 288: cluster mode
+constexpr int kClusterThreads = 12 * 32;                // 384: cluster mode (3 warpgroups; warps 9-11 only mirror barriers)
+// Many-row mode moves registers between warpgroups (setmaxnreg): the filter
+// warpgroups take kFilterRegs per thread, the finisher / producer warpgroups
+// give up to kOtherRegs. The block is launched with 128 per thread (512 x 128
+// = the whole register file), and 2 x 160 + 2 x 96 = 4 x 128, so the split is
+// exactly the launch allocation; the host enables it only after checking that
+// every kernel instance was built with 128 registers per thread.
+// Cluster mode does the same with three warpgroups: 2 x 160 + 64 = 3 x 128.
+constexpr int kLaunchRegs = 128, kFilterRegs = 160, kOtherRegs = 96, kMirrorRegs = 64;
+static_assert(2 * kFilterRegs + 2 * kOtherRegs == 4 * kLaunchRegs && kThreads * kLaunchRegs == 65536,
+              "the register split must equal the launch allocation");
+static_assert(2 * kFilterRegs + kMirrorRegs == 3 * kLaunchRegs && kClusterThreads == 3 * 128,
+              "the cluster-mode register split must equal the launch allocation");
 constexpr int kGroups = 8;                              // groups of 4 values per lane and stage
 constexpr int kVals = 4 * kGroups;                      // 32 values per lane and stage
 constexpr int kWarpElems = 32 * kVals;                  // 1024 per warp and stage
@@ -87,7 +99,6 @@ constexpr int kBigBucket = 64;                          // finisher: larger buck
 constexpr int kSmallBucket = 16;                        // finisher: largest bucket ranked by direct counting
 constexpr int kSortPasses = 3;                          // finisher: bucket count passes, at most
 constexpr int kBucketMax = 4096;                        // finisher bucket counters
-constexpr uint32_t kAbortBit = 0x80000000u;             // flag bit beside a published stage count
 constexpr uint32_t kUnsorted = DSA_FLAG_UNSORTED;
 
 template <class T>
@@ -112,6 +123,7 @@ struct Params {
   const int32_t* table;  // optional index table: out = table[row * table_stride + idx]
   int64_t table_stride;
   int32_t* out;
+  uint32_t regsplit;  // many-row mode: move registers between warpgroups (see kFilterRegs)
 };
 
 struct __align__(128) Smem {
@@ -143,7 +155,8 @@ struct __align__(128) Smem {
   uint32_t own_key;
   int32_t own_len;
   float row_t0;        // the current row's initial threshold
-  uint32_t abort;      // raised by the first pipeline wait that gives up
+  WaitCtl wait;        // abort flag and time limit of every pipeline wait
+  uint32_t abort_seen; // the abort flag as thread 0 read it before an item's last filter barrier
   uint32_t abort_any;  // cluster mode: some rank gave up (read by the leader)
   uint32_t final_bar;  // cluster mode: number of cluster barriers of the merge (0: not yet known)
   unsigned long long full[kMaxStages], empty[kMaxStages];
@@ -287,9 +300,8 @@ __device__ __forceinline__ void digit_histogram(uint32_t* hist, int n, V v, P pr
 
 // need-th largest of v(e) over the candidates with pred(e) (1 <= need <= their
 // number). Radix rounds over 8-bit windows below the highest bit where the
-// bounds differ; after each round the bounds shrink to the smallest and
-// largest value actually inside the chosen bucket (a bucket of one tied value
-// ends the search there). A bucket of <= 32 values is finished by one warp.
+// bounds differ; a bucket of <= 32 values is finished by one warp. Each thread
+// adds a run of equal digits with one atomic.
 template <class V, class P>
 __device__ uint32_t filter_kth(Smem& s, int n, uint32_t need, V v, P pred, int tid) {
   const int w = tid >> 5, lane = tid & 31;
@@ -307,7 +319,22 @@ __device__ uint32_t filter_kth(Smem& s, int n, uint32_t need, V v, P pred, int t
       s.bc[2] = 0u;
     }
     bar_filter();
-    digit_histogram(s.hist, n, v, pred, lo, hi, sh, tid);
+    {
+      uint32_t cur = 0xFFFFFFFFu, run = 0;
+      for (int e = tid; e < n; e += kFilterThreads) {
+        if (!pred(e)) continue;
+        const uint32_t x = v(e);
+        if (x < lo || x > hi) continue;
+        const uint32_t d = (x >> sh) & 255u;
+        if (d != cur) {
+          if (run) atomicAdd(&s.hist[cur], run);
+          cur = d;
+          run = 0;
+        }
+        ++run;
+      }
+      if (run) atomicAdd(&s.hist[cur], run);
+    }
     bar_filter();
     if (w == 0) find_bucket_warp0(s.hist, need, s.bc, lane);
     bar_filter();
@@ -335,9 +362,6 @@ __device__ uint32_t filter_kth(Smem& s, int n, uint32_t need, V v, P pred, int t
       }
       bar_filter();
       lo = hi = s.bc[3];
-    } else if (lo != hi) {
-      const uint32_t a = lo, b = hi;
-      filter_minmax(s, n, v, [&](int e) { return pred(e) && v(e) >= a && v(e) <= b; }, lo, hi, tid);
     }
     bar_filter();
   }
@@ -620,11 +644,8 @@ __device__ __forceinline__ Filter take_stage_split(Smem& s, Filter f, const uint
 }
 
 // Takes one stage after the filter barrier that completed its per-warp counts.
-// Returns false, writing nothing, when a warp flagged that its wait for the
-// stage gave up (kAbortBit of its count): every filter warp sees the same
-// counts, so all of them leave together.
 template <class T, bool kRing>
-__device__ __forceinline__ bool take_stage(Smem& s, Filter& f, const uint4* red, const T* src, uint32_t msk,
+__device__ __forceinline__ void take_stage(Smem& s, Filter& f, const uint4* red, const T* src, uint32_t msk,
                                            uint32_t idx0, int m, int tid) {
   const int w = tid >> 5, lane = tid & 31;
   uint32_t r[4 * ((kFilterWarps + 3) / 4)];
@@ -636,29 +657,24 @@ __device__ __forceinline__ bool take_stage(Smem& s, Filter& f, const uint4* red,
     r[4 * i + 2] = q.z;
     r[4 * i + 3] = q.w;
   }
-  uint32_t before = 0, tot = 0, flags = 0;
+  uint32_t before = 0, tot = 0;
 #pragma unroll
   for (int i = 0; i < kFilterWarps; ++i) {
     before += i < w ? r[i] : 0u;
     tot += r[i];
-    flags |= r[i];
   }
-  if (flags & kAbortBit) return false;
   if (f.cnt + tot <= static_cast<uint32_t>(kFiltCap)) {
     put_survivors<T, kRing>(s, src, msk, idx0, f.cnt + before, w, lane);
     f.cnt += tot;
   } else {
     f = take_stage_split<T, kRing>(s, f, reinterpret_cast<const uint32_t*>(red), src, msk, idx0, m, tid);
   }
-  return true;
 }
 
-// Publishes this warp's survivor count (read after the next filter barrier),
-// with kAbortBit set when a lane's wait for the stage gave up.
-__device__ __forceinline__ void publish(uint4* red, uint32_t msk, int w, int lane, bool fail) {
+// Publishes this warp's survivor count (read after the next filter barrier).
+__device__ __forceinline__ void publish(uint4* red, uint32_t msk, int w, int lane) {
   const uint32_t wt = __reduce_add_sync(kFull, __popc(msk));
-  const bool ab = __any_sync(kFull, fail);
-  if (lane == 0) reinterpret_cast<uint32_t*>(red)[w] = wt | (ab ? kAbortBit : 0u);
+  if (lane == 0) reinterpret_cast<uint32_t*>(red)[w] = wt;
 }
 
 __device__ __forceinline__ uint32_t stage_mask(const float (&v)[kVals], float t, bool edge, int64_t sj0, int64_t L,
@@ -698,7 +714,7 @@ __device__ __forceinline__ Filter refilter_from_global(Smem& s, Filter f, RowSpa
       for (int i = 0; i < 4; ++i) v[4 * q + i] = x[i];
     }
     const uint32_t msk = stage_mask(v, f.t, st == 0 || st + 1 == sp.nst, sj0, L, w, lane);
-    publish(&s.red[f.par][0], msk, w, lane, false);
+    publish(&s.red[f.par][0], msk, w, lane);
     bar_filter();
     take_stage<T, false>(s, f, &s.red[f.par][0], src, msk, base + static_cast<uint32_t>(sj0), m, tid);
     f.par ^= 1;
@@ -740,18 +756,6 @@ __device__ __noinline__ float sample_threshold(Smem& s, const T* row, int64_t L,
   return (T0 == 0u || T0 >= kInfKey) ? __int_as_float(0xff800000) : from_key(T0);
 }
 
-template <class T>
-__device__ __forceinline__ void load_slot(const Smem& s, int slot, int w, int lane, float (&v)[kVals]) {
-  const T* ring = reinterpret_cast<const T*>(s.ring) + slot * kStageElems;
-#pragma unroll
-  for (int q = 0; q < kGroups; ++q) {
-    float x[4];
-    Elem<T>::four(ring + w * kWarpElems + q * 128 + lane * 4, x);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) v[4 * q + i] = x[i];
-  }
-}
-
 // Consumer position in the ring.
 struct RingPos {
   int slot;        // ring slot of the next stage
@@ -761,24 +765,41 @@ struct RingPos {
 
 // Streams one item (a row, or a rank's chunk of a row: L entries whose stored
 // indices are base + item index) through the ring into the candidate buffer,
-// starting from threshold f.t. Returns false when a wait gave up; the filter
-// warps then leave together.
+// starting from threshold f.t. A stage whose wait gave up counts as empty:
+// after a timeout every wait of the CTA fails at once, so the loop runs out
+// quickly through the same barriers as always, and the caller learns of it
+// from the CTA's abort flag (a consensus at the next row or merge).
 template <class T>
-__device__ __forceinline__ bool stream_item(Smem& s, Filter& f, RingPos& rp, const RowSpan& sp, int32_t L, uint32_t base,
+__device__ __forceinline__ void stream_item(Smem& s, Filter& f, RingPos& rp, const RowSpan& sp, int32_t L, uint32_t base,
                                             int m, int tid) {
   constexpr int kStages = stages_of<T>();
   const int w = tid >> 5, lane = tid & 31;
   int32_t sj0 = static_cast<int32_t>(sp.j0);  // item index of the stage's first element (< L <= INT32_MAX)
   for (int st = 0; st < sp.nst; ++st, sj0 += kStageElems) {
-    const bool ok = mbar_wait(&s.full[rp.slot], rp.phase, &s.abort);
-    float v[kVals];
-    load_slot<T>(s, rp.slot, w, lane, v);  // values of a stage that never came are unused
-    const uint32_t msk = stage_mask(v, f.t, st == 0 || st + 1 == sp.nst, sj0, L, w, lane);
-    publish(&s.red[rp.par][0], msk, w, lane, !ok);
+    const bool ok = mbar_wait(&s.full[rp.slot], rp.phase, &s.wait);
+    // the pass mask, group by group as the values are loaded (values of a
+    // stage that never came are unused)
+    uint32_t msk = 0;
+    {
+      const T* rg = reinterpret_cast<const T*>(s.ring) + rp.slot * kStageElems + w * kWarpElems + lane * 4;
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q) {
+        float x[4];
+        Elem<T>::four(rg + q * 128, x);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) msk |= static_cast<uint32_t>(!(x[i] < f.t)) << (4 * q + i);
+      }
+      if (st == 0 || st + 1 == sp.nst) {
+        int lo, hi;
+        stage_bounds(sj0, L, lo, hi);
+        msk &= range_mask(w, lane, lo, hi);
+      }
+      if (!ok) msk = 0u;
+    }
+    publish(&s.red[rp.par][0], msk, w, lane);
     bar_filter();  // every warp's count of this stage is published
     const T* ring = reinterpret_cast<const T*>(s.ring) + rp.slot * kStageElems;
-    if (!take_stage<T, true>(s, f, &s.red[rp.par][0], ring, msk, base + static_cast<uint32_t>(sj0), m, tid))
-      return false;
+    take_stage<T, true>(s, f, &s.red[rp.par][0], ring, msk, base + static_cast<uint32_t>(sj0), m, tid);
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.empty[rp.slot]);
     if (f.cnt > static_cast<uint32_t>(kTrigger)) compact_any(s, f, m, tid);
@@ -789,8 +810,10 @@ __device__ __forceinline__ bool stream_item(Smem& s, Filter& f, RingPos& rp, con
       rp.phase ^= 1u;
     }
   }
+  // a snapshot of the abort flag, the same for every filter thread after the
+  // barrier (the flag itself may be raised by another role at any time)
+  if (tid == 0) s.abort_seen = *reinterpret_cast<volatile uint32_t*>(&s.wait.abort);
   bar_filter();  // every append is visible
-  return true;
 }
 
 template <class T>
@@ -805,6 +828,7 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
   int64_t row = blockIdx.x;
   int32_t L_next = row < p.num_rows ? static_cast<int32_t>(clamp_len(p.lengths, row, p.row_stride)) : 0;
   for (; row < p.num_rows; row += gridDim.x, ++h) {
+    if (s.abort_seen) return;  // a wait gave up during the previous row: the filter warps leave together
     const int32_t L = L_next;  // lengths are int32, so is every clamped length
     if (row + gridDim.x < p.num_rows)
       L_next = static_cast<int32_t>(clamp_len(p.lengths, row + gridDim.x, p.row_stride));
@@ -835,8 +859,8 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
     f.compacted = false;
     f.strict = false;
     f.bounded = false;
-    if (!stream_item<T>(s, f, rp, sp, L, 0u, m, tid)) return;  // a wait gave up: nothing is handed over
-    const bool reread = spec && !f.compacted && f.cnt < static_cast<uint32_t>(m);
+    stream_item<T>(s, f, rp, sp, L, 0u, m, tid);
+    const bool reread = spec && !f.compacted && f.cnt < static_cast<uint32_t>(m) && !s.abort_seen;
     if (reread) {
       if (tid == 0) atomicOr(&g_status, kStatusReread);
       f = refilter_from_global<T>(s, f, sp, L, 0u, m, tid);
@@ -856,9 +880,9 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
       }
     }
     bar_filter();  // the own estimate is read at the next row's start
-    // hand over: wait until the finishers released the previous handover
-    const bool ok = mbar_wait_sleep(&s.hempty, (h & 1) ^ 1, &s.abort);
-    if (bar_filter_any(!ok)) return;
+    // hand over: wait until the finishers released the previous handover (a
+    // wait that gave up hands over regardless; the row's output is undefined)
+    mbar_wait_sleep(&s.hempty, (h & 1) ^ 1, &s.wait);
     for (int e = tid; e < static_cast<int>(f.cnt); e += kFilterThreads) {
       s.hkey[e] = s.fkey[e];
       s.hidx[e] = s.fidx[e];
@@ -903,54 +927,255 @@ struct Finisher {
     return sh;
   }
 
-  // index -> output value: the optional table maps a row-local index to the
-  // caller's value (-1 passes through)
-  __device__ __forceinline__ static int32_t emit(const Params& p, int64_t row, int32_t idx) {
-    if (p.table == nullptr || idx < 0) return idx;
-    return __ldg(p.table + row * p.table_stride + idx);
-  }
-
-  // Candidates [0, n) ordered in place by (key descending, index ascending)
-  // with a bitonic network over the next power of two (padding keys 0 sort
-  // last), then the first m written. Ends with a barrier.
-  __device__ __noinline__ static void finish_sorted(Smem& s, int n, int m, int k, int64_t row, const Params& p,
-                                                    int fid) {
-    int32_t* o = p.out + row * static_cast<int64_t>(k);
-    int N = 1;
-    while (N < n) N <<= 1;
-    for (int e = n + fid; e < N; e += NT) {
-      s.hkey[e] = 0u;
-      s.hidx[e] = 0xFFFFFFFFu;
-    }
-    bar();
-    for (int size = 2; size <= N; size <<= 1) {
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int t = fid; t < (N >> 1); t += NT) {
-          const int i = 2 * t - (t & (stride - 1));
-          const int j = i + stride;
-          const uint32_t ki = s.hkey[i], ii = s.hidx[i], kj = s.hkey[j], ij = s.hidx[j];
-          const bool j_first = kj > ki || (kj == ki && ij < ii);  // j belongs before i
-          if (j_first == ((i & size) == 0)) {
-            s.hkey[i] = kj;
-            s.hidx[i] = ij;
-            s.hkey[j] = ki;
-            s.hidx[j] = ii;
-          }
+  // Ranks, position-parallel (used when the finisher runs alone, where its
+  // latency is the kernel's tail): each warp takes 32 consecutive positions
+  // of the bucket order (one per lane) up to the end of the bucket holding
+  // rank m-1. A candidate's rank is its bucket's start plus the bucket members
+  // that beat it; members in the same 32-position window come from the
+  // neighbouring lanes by shuffles (only as far as the widest bucket of the
+  // window), the few beyond the window from shared memory. In set mode only
+  // the bucket holding rank m-1 is ranked; earlier positions stay as they lie.
+  __device__ __forceinline__ static void rank_by_windows(Smem& s, int n, int m, int k, int a, uint32_t bm,
+                                                         bool set_mode, uint32_t kmax, int sh, int fid) {
+    const int fw = fid >> 5, lane = fid & 31;
+    const uint32_t qend = s.bcnt[bm];  // positions past this have rank >= m
+    const uint32_t cut0 = bm ? s.bcnt[bm - 1] : 0u;
+    for (uint32_t q0 = static_cast<uint32_t>(fw) * 32u; q0 < qend; q0 += kWarps * 32u) {
+      const uint32_t q = q0 + lane;
+      const bool v = q < qend;
+      const uint32_t e = v ? s.perm[q] : 0u;
+      const uint32_t key = v ? s.hkey[e] : 0u, idx = v ? s.hidx[e] : 0xFFFFFFFFu;
+      uint32_t s0 = q, s1 = q + 1;  // invalid lanes: a bucket of their own
+      if (v) {
+        const uint32_t b =
+            static_cast<uint32_t>((((static_cast<uint64_t>(kmax - key)) << 32) | idx) >> sh);
+        s0 = b ? s.bcnt[b - 1] : 0u;
+        s1 = s.bcnt[b];
+      }
+      uint32_t r = 0;
+      const bool need = v && !(set_mode && s1 <= cut0) && s0 < static_cast<uint32_t>(m) && s1 - s0 > 1u;
+      const uint32_t span = __reduce_max_sync(kFull, need ? s1 - s0 : 1u);
+      for (uint32_t d = 1; d < span && d < 32u; ++d) {
+        const uint32_t ku = __shfl_down_sync(kFull, key, d), iu = __shfl_down_sync(kFull, idx, d);
+        const uint32_t kd = __shfl_up_sync(kFull, key, d), id = __shfl_up_sync(kFull, idx, d);
+        if (need) {
+          if (lane + d < 32u && q + d < s1) r += ku > key || (ku == key && iu < idx);
+          if (lane >= d && q - d >= s0) r += kd > key || (kd == key && id < idx);
         }
-        bar();
+      }
+      if (need && (s0 < q0 || s1 > q0 + 32u)) {  // bucket members outside the window
+        for (uint32_t q2 = s0; q2 < s1; ++q2) {
+          if (q2 >= q0 && q2 < q0 + 32u) continue;
+          const uint32_t j = s.perm[q2];
+          const uint32_t kj = s.hkey[j], ij = s.hidx[j];
+          r += kj > key || (kj == key && ij < idx);
+        }
+      }
+      if (v) {
+        const uint32_t pos = (set_mode && s1 <= cut0) ? q : s0 + r;
+        if (pos < static_cast<uint32_t>(m)) {
+          s.ostage[pos] = static_cast<int32_t>(idx);
+          if (pos == static_cast<uint32_t>(k - 1)) s.rec[0] = key;
+          if (pos == static_cast<uint32_t>(a)) s.rec[1] = key;
+        }
       }
     }
+  }
+
+  // Writes o[0 .. m) from the staged indices; the optional table maps a
+  // row-local index to the caller's value (-1 passes through). With a table,
+  // each thread first
+  // issues eight independent table loads, then stores: the gathers overlap
+  // instead of waiting one by one.
+  __device__ __forceinline__ static void write_out(const int32_t* staged, int32_t* o, int m, int64_t row,
+                                                   const Params& p, int fid) {
+    if (p.table == nullptr) {
+      for (int q = fid; q < m; q += NT) o[q] = staged[q];
+      return;
+    }
+    const int32_t* trow = p.table + row * p.table_stride;
+    for (int q0 = fid; q0 < m; q0 += 8 * NT) {
+      int32_t v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int q = q0 + u * NT;
+        const int32_t idx = q < m ? staged[q] : -1;
+        v[u] = idx >= 0 ? __ldg(trow + idx) : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (q0 + u * NT < m) o[q0 + u * NT] = v[u];
+    }
+  }
+
+  // Candidates [0, n) ordered by the composite C = (kmax - key) << 32 | index
+  // (key descending, index ascending) with a stable LSD radix sort of a
+  // 16-bit permutation, one counting pass per byte of C that differs between
+  // candidates (values on a coarse grid leave most key bytes equal), then the
+  // first m written. Used when buckets stay crowded with equal keys, where
+  // counting ranks inside a bucket would be quadratic. Ends with a barrier.
+  //   per pass: each warp owns a contiguous range of the current order and
+  //   walks it 32 at a time; lanes holding the same digit are matched with
+  //   eight ballots; per-warp digit counts are scanned digit-major, warp-minor,
+  //   so the scatter keeps the current order among equal digits.
+  __device__ __noinline__ static void finish_sorted(Smem& s, int n, int m, int k, uint32_t kmax, int64_t row,
+                                                    const Params p, int fid) {
+    const int fw = fid >> 5, lane = fid & 31;
+    int32_t* o = p.out + row * static_cast<int64_t>(k);
+    uint16_t* pa = s.perm;
+    uint16_t* pb = reinterpret_cast<uint16_t*>(s.ostage);  // 2 x kMaxK bytes = kHandCap entries
+    uint32_t* cnt = s.bcnt;                                // [kWarps][256] per-warp digit counts
+    uint32_t* dbase = s.bcnt + kWarps * 256;               // [256] digit starts
+    // bytes of C that vary: from the OR and AND of its two halves
+    uint32_t or_hi = 0u, and_hi = 0xFFFFFFFFu, or_lo = 0u, and_lo = 0xFFFFFFFFu;
+    for (int e = fid; e < n; e += NT) {
+      const uint32_t hi = kmax - s.hkey[e], lo = s.hidx[e];
+      or_hi |= hi;
+      and_hi &= hi;
+      or_lo |= lo;
+      and_lo &= lo;
+      pa[e] = static_cast<uint16_t>(e);
+    }
+    or_hi = __reduce_or_sync(kFull, or_hi);
+    and_hi = __reduce_and_sync(kFull, and_hi);
+    or_lo = __reduce_or_sync(kFull, or_lo);
+    and_lo = __reduce_and_sync(kFull, and_lo);
+    if (lane == 0) {
+      s.nred[0][fw] = or_hi;
+      s.nred[1][fw] = and_hi;
+      s.nred[2][fw] = or_lo;
+      s.nred[3][fw] = and_lo;
+    }
+    bar();
+    uint32_t vhi = 0u, vlo = 0u;
+    {
+      uint32_t a0 = 0u, a1 = 0xFFFFFFFFu, b0 = 0u, b1 = 0xFFFFFFFFu;
+#pragma unroll
+      for (int ww = 0; ww < kWarps; ++ww) {
+        a0 |= s.nred[0][ww];
+        a1 &= s.nred[1][ww];
+        b0 |= s.nred[2][ww];
+        b1 &= s.nred[3][ww];
+      }
+      vhi = a0 & ~a1;
+      vlo = b0 & ~b1;
+    }
+    const int per = ((n + kWarps - 1) / kWarps + 31) & ~31;  // items per warp, whole chunks
+    const int i0 = fw * per, i1 = min(n, i0 + per);
+    const uint32_t lt = lanemask_lt();
+    for (int byte = 0; byte < 8; ++byte) {
+      const uint32_t vary = byte < 4 ? (vlo >> (8 * byte)) & 255u : (vhi >> (8 * (byte - 4))) & 255u;
+      if (vary == 0u) continue;  // the same in every candidate: the pass would be the identity
+      const int sh = 8 * (byte & 3);
+      const bool hi_half = byte >= 4;
+      for (int d = lane; d < 256; d += 32) cnt[fw * 256 + d] = 0u;
+      __syncwarp();
+      // count
+      for (int c0 = i0; c0 < i1; c0 += 32) {
+        const int i = c0 + lane;
+        const bool v = i < i1;
+        uint32_t d = 0u;
+        if (v) {
+          const uint32_t e = pa[i];
+          d = ((hi_half ? kmax - s.hkey[e] : s.hidx[e]) >> sh) & 255u;
+        }
+        uint32_t peers = __ballot_sync(kFull, v);
+#pragma unroll
+        for (int bit = 0; bit < 8; ++bit) {
+          const uint32_t bb = __ballot_sync(kFull, (d >> bit) & 1u);
+          peers &= ((d >> bit) & 1u) ? bb : ~bb;
+        }
+        if (v && (peers & lt) == 0u) cnt[fw * 256 + d] += __popc(peers);
+        __syncwarp();
+      }
+      bar();
+      // digit starts: digit-major, warp-minor exclusive prefix
+      for (int d = fid; d < 256; d += NT) {
+        uint32_t t = 0;
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) t += cnt[ww * 256 + d];
+        dbase[d] = t;
+      }
+      bar();
+      if (fw == 0) {
+        uint32_t c[8], sum = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          c[t] = dbase[8 * lane + t];
+          sum += c[t];
+        }
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o2 = 1; o2 < 32; o2 <<= 1) {
+          const uint32_t y = __shfl_up_sync(kFull, incl, o2);
+          if (lane >= o2) incl += y;
+        }
+        uint32_t run = incl - sum;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          dbase[8 * lane + t] = run;
+          run += c[t];
+        }
+      }
+      bar();
+      for (int d = fid; d < 256; d += NT) {
+        uint32_t run = dbase[d];
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) {
+          const uint32_t t = cnt[ww * 256 + d];
+          cnt[ww * 256 + d] = run;
+          run += t;
+        }
+      }
+      bar();
+      // scatter in order
+      for (int c0 = i0; c0 < i1; c0 += 32) {
+        const int i = c0 + lane;
+        const bool v = i < i1;
+        uint32_t d = 0u, e = 0u;
+        if (v) {
+          e = pa[i];
+          d = ((hi_half ? kmax - s.hkey[e] : s.hidx[e]) >> sh) & 255u;
+        }
+        uint32_t peers = __ballot_sync(kFull, v);
+#pragma unroll
+        for (int bit = 0; bit < 8; ++bit) {
+          const uint32_t bb = __ballot_sync(kFull, (d >> bit) & 1u);
+          peers &= ((d >> bit) & 1u) ? bb : ~bb;
+        }
+        const uint32_t base = v ? cnt[fw * 256 + d] : 0u;
+        if (v) pb[base + __popc(peers & lt)] = static_cast<uint16_t>(e);
+        __syncwarp();
+        if (v && (peers & lt) == 0u) cnt[fw * 256 + d] = base + __popc(peers);
+        __syncwarp();
+      }
+      bar();
+      uint16_t* t = pa;
+      pa = pb;
+      pb = t;
+    }
     const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
-    for (int q = fid; q < m; q += NT) {
-      o[q] = emit(p, row, static_cast<int32_t>(s.hidx[q]));
-      if (q == k - 1) s.rec[0] = s.hkey[q];
-      if (q == a) s.rec[1] = s.hkey[q];
+    if (fid == 0) {
+      if (m == k) s.rec[0] = s.hkey[pa[k - 1]];
+      if (a < m) s.rec[1] = s.hkey[pa[a]];
+    }
+    // the sorted order's first m indices (the permutation buffer may be the
+    // output stage, so it is read, not staged)
+    if (p.table == nullptr) {
+      for (int q = fid; q < m; q += NT) o[q] = static_cast<int32_t>(s.hidx[pa[q]]);
+    } else {
+      const int32_t* trow = p.table + row * p.table_stride;
+      for (int q = fid; q < m; q += NT) o[q] = __ldg(trow + s.hidx[pa[q]]);
     }
     bar();
   }
 
   // Ranks n candidates and writes the row: m indices, then -1 up to k.
-  __device__ __noinline__ static void finish(Smem& s, int n, int m, int k, int64_t row, const Params& p, int fid) {
+  // `alone`: nothing else runs on the SM meanwhile (a CTA's last row, a
+  // cluster's leader).
+  // (Inlined into the finisher warps' loop; a call there cost a few percent.)
+  __device__ __forceinline__ static void finish(Smem& s, int n, int m, int k, int64_t row, const Params& p, int fid,
+                                                bool alone) {
     const int fw = fid >> 5, lane = fid & 31;
     int32_t* o = p.out + row * static_cast<int64_t>(k);
     for (int q = m + fid; q < k; q += NT) o[q] = -1;
@@ -1055,7 +1280,7 @@ struct Finisher {
     if (big > static_cast<uint32_t>(kBigBucket)) {
       // many candidates share a bucket (values on a coarse grid): counting
       // ranks inside it would be quadratic, so sort everything instead
-      finish_sorted(s, n, m, k, row, p, fid);
+      finish_sorted(s, n, m, k, kmax, row, p, fid);
       return;
     }
     for (int e = fid; e < n; e += NT) {
@@ -1066,10 +1291,16 @@ struct Finisher {
     }
     bar();  // bcnt[b] is now the end of bucket b (= start of b + 1)
     const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
-    if (p.flags & kUnsorted) {
+    const uint32_t bm = s.bc[4];
+    const bool set_mode = (p.flags & kUnsorted) != 0u;
+    if (alone && n > 2 * m) {
+      // nothing overlaps this row, and most candidates rank past m: ranking
+      // only the positions before m is fastest (the per-candidate loop below
+      // takes the fewest issue slots, which counts while rows still stream)
+      rank_by_windows(s, n, m, k, a, bm, set_mode, kmax, sh, fid);
+    } else if (set_mode) {
       // set mode: positions before the bucket holding rank m-1 are taken as
       // they lie (bucket order); only that bucket's members are ranked
-      const uint32_t bm = s.bc[4];
       const uint32_t s0 = bm ? s.bcnt[bm - 1] : 0u, s1 = s.bcnt[bm];
       for (uint32_t q = fid; q < s0; q += NT) {
         const uint32_t e = s.perm[q];
@@ -1092,6 +1323,7 @@ struct Finisher {
         }
       }
     } else {
+      // each candidate: its bucket's start plus the bucket members ahead of it
       for (int e = fid; e < n; e += NT) {
         const uint32_t key = s.hkey[e], idx = s.hidx[e];
         const uint64_t cc = comp(key, idx);
@@ -1113,30 +1345,43 @@ struct Finisher {
       }
     }
     bar();
-    for (int q = fid; q < m; q += NT) o[q] = emit(p, row, s.ostage[q]);
+    write_out(s.ostage, o, m, row, p, fid);
   }
 };
 
 using RowFinisher = Finisher<kFinishThreads, 2>;
 using LeaderFinisher = Finisher<kFilterThreads, 1>;
 
+// The estimate the filter starts a later row from: the k-th value minus half
+// the gap to the 3k/4-th, and at least one step of the element type's value
+// grid below the k-th (a coarse grid, such as bf16 logits, often puts both
+// ranks on one value; an estimate equal to the k-th value then lets too few
+// values of a similar row through and forces a re-read).
+template <class T>
+__device__ __forceinline__ float row_estimate(float vt, float va) {
+  constexpr int kMantissa = sizeof(T) == 4 ? 23 : (Elem<T>::kCode == DSA_DTYPE_BF16 ? 7 : 10);
+  const float step = fabsf(vt) * (1.0f / static_cast<float>(1 << kMantissa));
+  return vt - fmaxf(0.5f * (va - vt), step);
+}
+
+template <class T>
 __device__ void finish_loop(Smem& s, const Params& p, int fid) {
   const int lane = fid & 31;
   const int k = p.k;
   int h = 0;
   for (int64_t row = blockIdx.x; row < p.num_rows; row += gridDim.x, ++h) {
-    const bool ok = mbar_wait_sleep(&s.hfull, h & 1, &s.abort);
+    const bool ok = mbar_wait_sleep(&s.hfull, h & 1, &s.wait);
     if (bar_any<2, kFinishThreads>(!ok)) return;  // the filter warps left: nothing more comes
     const int n = s.h_n, m = s.h_m;
     const int64_t L = s.h_len;
-    RowFinisher::finish(s, n, m, k, s.h_row, p, fid);
+    RowFinisher::finish(s, n, m, k, s.h_row, p, fid, row + gridDim.x >= p.num_rows);
     if (fid == 0) {
       bool est_ok = false;
       float e = 0.f;
       if (n > 0 && m == k) {
         const uint32_t kt = s.rec[0], ka = s.rec[1];
         const float vt = from_key(kt), va = from_key(ka);
-        e = vt - 0.5f * (va - vt);
+        e = row_estimate<T>(vt, va);
         est_ok = kt != kNanKey && ka != kNanKey && isfinite(e);
       }
       s.est[h & 1] = e;
@@ -1157,7 +1402,7 @@ __device__ __forceinline__ bool produce_span(Smem& s, const RowSpan& sp, int& sl
   constexpr int kStages = stages_of<T>();
   constexpr uint32_t kStageBytes = kStageElems * sizeof(T);
   for (int st = 0; st < sp.nst; ++st, ++gi) {
-    if (!mbar_wait_sleep(&s.empty[slot], phase ^ 1u, &s.abort)) return false;
+    if (!mbar_wait_sleep(&s.empty[slot], phase ^ 1u, &s.wait)) return false;
     if (gi != skip) {
       const uint32_t bytes = st + 1 == sp.nst ? sp.last_bytes : kStageBytes;
       fence_proxy_async();
@@ -1180,7 +1425,7 @@ __device__ __forceinline__ bool produce_span(Smem& s, const RowSpan& sp, int& sl
 // never exits with a bulk copy still writing into its shared memory.
 __device__ __forceinline__ void producer_drain(Smem& s, uint32_t armed, uint32_t arm_par) {
   for (int i = 0; i < kMaxStages; ++i)
-    if ((armed >> i) & 1u) mbar_drain(&s.full[i], (arm_par >> i) & 1u);
+    if ((armed >> i) & 1u) mbar_drain(&s.full[i], (arm_par >> i) & 1u, &s.wait);
 }
 
 template <class T>
@@ -1356,52 +1601,74 @@ __device__ __noinline__ uint32_t cluster_merge(Smem& s, uint32_t n_r, uint32_t m
   return total;
 }
 
-template <class T>
-__device__ __noinline__ void cluster_row(Smem& s, const Params& p, int tid) {
-  const int w = tid >> 5, lane = tid & 31;  // warp kClusterWarp is the producer
-  const uint32_t rank = cluster_rank(), ncta = cluster_size();
-  const int64_t row = cluster_index();
-  const T* rowp = static_cast<const T*>(p.logits) + row * p.row_stride;
-  const int64_t L = clamp_len(p.lengths, row, p.row_stride);
-  const int k = p.k;
-  const uint32_t m = static_cast<uint32_t>(min64(k, L));
-  if (m == 0) {  // the same for every CTA of the cluster: no merge, no barrier
-    if (rank == 0 && w < kFilterWarps)
-      for (int q = tid; q < k; q += kFilterThreads) p.out[row * static_cast<int64_t>(k) + q] = -1;
-    return;
-  }
-  int64_t chunk = (L + ncta - 1) / ncta;
+// The row and chunk of this CTA in cluster mode (the same computation in every
+// role of every rank).
+struct ClusterItem {
+  uint32_t rank, ncta;
+  int64_t row, L, c0, c1;
+  uint32_t m;
+};
+
+__device__ __forceinline__ ClusterItem cluster_item(const Params& p) {
+  ClusterItem it;
+  it.rank = cluster_rank();
+  it.ncta = cluster_size();
+  it.row = cluster_index();
+  it.L = clamp_len(p.lengths, it.row, p.row_stride);
+  it.m = static_cast<uint32_t>(min64(p.k, it.L));
+  int64_t chunk = (it.L + it.ncta - 1) / it.ncta;
   chunk = (chunk + 7) & ~static_cast<int64_t>(7);
-  const int64_t c0 = min64(L, static_cast<int64_t>(rank) * chunk);
-  const int64_t c1 = min64(L, c0 + chunk);
-  const int32_t Lc = static_cast<int32_t>(c1 - c0);
-  const RowSpan sp = row_span(rowp + c0, Lc);
-  if (w == kClusterWarp) {
-    // producer: lane 0 streams the chunk; then the whole warp mirrors the
-    // merge's cluster barriers, leaving after the last one
-    if (lane == 0) {
-      int slot = 0;
-      uint32_t phase = 0u, armed = 0u, arm_par = 0u;
-      long long gi = 0;
-      produce_span<T>(s, sp, slot, phase, gi, g_skip_stage, armed, arm_par);
-      producer_drain(s, armed, arm_par);
-    }
-    __syncwarp();
-    for (uint32_t i = 1;; ++i) {
-      cluster_barrier();
-      const volatile uint32_t* fb = &s.final_bar;
-      if (*fb == i) break;
-    }
+  it.c0 = min64(it.L, static_cast<int64_t>(it.rank) * chunk);
+  it.c1 = min64(it.L, it.c0 + chunk);
+  return it;
+}
+
+// Cluster mode, warps kClusterWarp.. (one warpgroup): lane 0 of the first
+// streams the chunk into the ring; then every warp of the group mirrors the
+// merge's cluster barriers (s.final_bar tells how many), leaving after the last.
+template <class T>
+__device__ __noinline__ void cluster_mirror(Smem& s, const Params p, int tid) {
+  const int w = tid >> 5, lane = tid & 31;
+  const ClusterItem it = cluster_item(p);
+  if (it.m == 0) return;  // the same for every CTA of the cluster: no merge, no barrier
+  if (w == kClusterWarp && lane == 0) {
+    const T* rowp = static_cast<const T*>(p.logits) + it.row * p.row_stride;
+    const RowSpan sp = row_span(rowp + it.c0, it.c1 - it.c0);
+    int slot = 0;
+    uint32_t phase = 0u, armed = 0u, arm_par = 0u;
+    long long gi = 0;
+    produce_span<T>(s, sp, slot, phase, gi, g_skip_stage, armed, arm_par);
+    producer_drain(s, armed, arm_par);
+  }
+  __syncwarp();
+  for (uint32_t i = 1;; ++i) {
+    cluster_barrier();
+    const volatile uint32_t* fb = &s.final_bar;
+    if (*fb == i) break;
+  }
+}
+
+// Cluster mode, filter warps: this rank's chunk, then the merge; the leader
+// ranks and writes the row.
+template <class T>
+__device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid) {
+  const ClusterItem it = cluster_item(p);
+  const int k = p.k;
+  if (it.m == 0) {  // the same for every CTA of the cluster: no merge, no barrier
+    if (it.rank == 0)
+      for (int q = tid; q < k; q += kFilterThreads) p.out[it.row * static_cast<int64_t>(k) + q] = -1;
     return;
   }
-  // filter warps: this rank's chunk, then the merge
-  const uint32_t m_r = min(m, static_cast<uint32_t>(Lc));
+  const T* rowp = static_cast<const T*>(p.logits) + it.row * p.row_stride;
+  const int32_t Lc = static_cast<int32_t>(it.c1 - it.c0);
+  const RowSpan sp = row_span(rowp + it.c0, Lc);
+  const uint32_t m_r = min(it.m, static_cast<uint32_t>(Lc));
   Filter f;
   f.par = 0;
   f.t = __int_as_float(0xff800000);
   bool spec = false;
   if (Lc >= kSampleMinLen && m_r > 0) {
-    const float ts = sample_threshold(s, rowp + c0, Lc, static_cast<int>(m_r), tid);
+    const float ts = sample_threshold(s, rowp + it.c0, Lc, static_cast<int>(m_r), tid);
     if (ts > __int_as_float(0xff800000)) {
       spec = true;
       f.t = ts;
@@ -1412,32 +1679,33 @@ __device__ __noinline__ void cluster_row(Smem& s, const Params& p, int tid) {
   f.strict = false;
   f.bounded = false;
   RingPos rp{0, 0u, 0u};
-  const bool ok = stream_item<T>(s, f, rp, sp, Lc, static_cast<uint32_t>(c0), static_cast<int>(m_r), tid);
+  stream_item<T>(s, f, rp, sp, Lc, static_cast<uint32_t>(it.c0), static_cast<int>(m_r), tid);
+  const bool ok = !s.abort_seen;
   if (!ok) {
     f.cnt = 0;  // no candidates from this rank; it still takes part in the merge
   } else {
     if (spec && !f.compacted && f.cnt < m_r) {
       if (tid == 0) atomicOr(&g_status, kStatusReread);
-      f = refilter_from_global<T>(s, f, sp, Lc, static_cast<uint32_t>(c0), static_cast<int>(m_r), tid);
+      f = refilter_from_global<T>(s, f, sp, Lc, static_cast<uint32_t>(it.c0), static_cast<int>(m_r), tid);
     }
     if (f.cnt > static_cast<uint32_t>(kHandCap)) compact_any(s, f, static_cast<int>(m_r), tid);
   }
-  const uint32_t total = cluster_merge(s, f.cnt, m, !ok, rank, ncta, tid);
-  if (rank != 0) return;
+  const uint32_t total = cluster_merge(s, f.cnt, it.m, !ok, it.rank, it.ncta, tid);
+  if (it.rank != 0) return;
   if (s.abort_any) {  // some rank gave up: no valid result for this row
-    for (int q = tid; q < k; q += kFilterThreads) p.out[row * static_cast<int64_t>(k) + q] = -1;
+    for (int q = tid; q < k; q += kFilterThreads) p.out[it.row * static_cast<int64_t>(k) + q] = -1;
     return;
   }
-  LeaderFinisher::finish(s, static_cast<int>(total), static_cast<int>(m), k, row, p, tid);
+  LeaderFinisher::finish(s, static_cast<int>(total), static_cast<int>(it.m), k, it.row, p, tid, true);
 }
 
 }  // namespace rows
 
 // Many rows (cluster size 1): grid = min(num_rows, SMs), one CTA per SM,
-// rows strided by the grid, 480 threads. A cluster per row: grid = num_rows *
-// cluster size, 288 threads.
+// rows strided by the grid, 512 threads. A cluster per row: grid = num_rows *
+// cluster size, 384 threads.
 template <class T>
-__global__ void __launch_bounds__(rows::kThreads, 1) topk_kernel(const rows::Params p) {
+__global__ void __launch_bounds__(rows::kThreads) topk_kernel(const rows::Params p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   rows::Smem& s = *reinterpret_cast<rows::Smem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1456,20 +1724,33 @@ __global__ void __launch_bounds__(rows::kThreads, 1) topk_kernel(const rows::Par
     }
     s.own_key = 0u;
     s.own_len = 0;
-    s.abort = 0u;
+    s.wait.abort = 0u;
+    s.abort_seen = 0u;
+    s.wait.limit_ns = g_wait_limit_ns;
     s.abort_any = 0u;
     s.final_bar = 0u;
     fence_mbar_init();
   }
   __syncthreads();
   pdl_enter();  // every thread: inputs and outputs are touched only after this
+  if (p.regsplit) {  // whole warpgroups: warps 0-7 filter; the rest finisher / producer / mirror
+    if (warp < rows::kFilterWarps)
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(rows::kFilterRegs) : "memory");
+    else if (!clustered)
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(rows::kOtherRegs) : "memory");
+    else
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(rows::kMirrorRegs) : "memory");
+  }
   if (clustered) {
-    rows::cluster_row<T>(s, p, tid);
+    if (warp < rows::kFilterWarps)
+      rows::cluster_filter<T>(s, p, tid);
+    else
+      rows::cluster_mirror<T>(s, p, tid);
   } else if (warp < rows::kFilterWarps) {
     rows::filter_loop<T>(s, p, tid);
   } else if (warp < rows::kProducerWarp) {
-    rows::finish_loop(s, p, tid - rows::kFilterThreads);
-  } else if (lane == 0) {
+    rows::finish_loop<T>(s, p, tid - rows::kFilterThreads);
+  } else if (warp == rows::kProducerWarp && lane == 0) {
     rows::produce_loop<T>(s, p);
   }
 }
