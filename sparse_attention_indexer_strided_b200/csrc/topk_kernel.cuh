@@ -54,6 +54,8 @@
 // over the indices of the tied keys) instead of a capped tie list.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace dsa {
@@ -1011,25 +1013,132 @@ struct Finisher {
     }
   }
 
+  // One stable LSD pass per BITS-bit digit over [lo_bit, hi_bit] of one half
+  // of C (half 0: the index, half 1: kmax - key), moving the permutation from
+  // *pa to *pb and swapping them. Counters are 32-bit where they fit beside
+  // the digit starts in the bucket-counter space, else 16-bit (n <= 4096).
+  template <int BITS>
+  __device__ __forceinline__ static void radix_passes(Smem& s, int n, uint32_t kmax, int half, uint32_t vary,
+                                                      uint16_t*& pa, uint16_t*& pb, int fid) {
+    constexpr int kBins = 1 << BITS;
+    using CT = typename std::conditional<(kWarps + 1) * kBins * 4 <= kBucketMax * 4, uint32_t, uint16_t>::type;
+    const int fw = fid >> 5, lane = fid & 31;
+    CT* cnt = reinterpret_cast<CT*>(s.bcnt);  // [kWarps][kBins] per-warp digit counts
+    uint32_t* dbase = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(s.bcnt) + kWarps * kBins * sizeof(CT));
+    const int per = ((n + kWarps - 1) / kWarps + 31) & ~31;  // items per warp, whole chunks
+    const int i0 = fw * per, i1 = min(n, i0 + per);
+    const uint32_t lt = lanemask_lt();
+    const int lo_bit = __ffs(vary) - 1, hi_bit = 31 - __clz(vary);
+    for (int sh = lo_bit; sh <= hi_bit; sh += BITS) {
+      for (int d = lane; d < kBins; d += 32) cnt[fw * kBins + d] = 0;
+      __syncwarp();
+      // count
+      for (int c0 = i0; c0 < i1; c0 += 32) {
+        const int i = c0 + lane;
+        const bool v = i < i1;
+        uint32_t d = 0u;
+        if (v) {
+          const uint32_t e = pa[i];
+          d = ((half ? kmax - s.hkey[e] : s.hidx[e]) >> sh) & (kBins - 1);
+        }
+        uint32_t peers = __ballot_sync(kFull, v);
+#pragma unroll
+        for (int bit = 0; bit < BITS; ++bit) {
+          const uint32_t bb = __ballot_sync(kFull, (d >> bit) & 1u);
+          peers &= ((d >> bit) & 1u) ? bb : ~bb;
+        }
+        if (v && (peers & lt) == 0u) cnt[fw * kBins + d] = static_cast<CT>(cnt[fw * kBins + d] + __popc(peers));
+        __syncwarp();
+      }
+      bar();
+      // digit starts: digit-major, warp-minor exclusive prefix
+      for (int d = fid; d < kBins; d += NT) {
+        uint32_t t = 0;
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) t += cnt[ww * kBins + d];
+        dbase[d] = t;
+      }
+      bar();
+      if (fw == 0) {
+        constexpr int kPer = kBins / 32;
+        uint32_t c[kPer], sum = 0;
+#pragma unroll
+        for (int t = 0; t < kPer; ++t) {
+          c[t] = dbase[kPer * lane + t];
+          sum += c[t];
+        }
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o2 = 1; o2 < 32; o2 <<= 1) {
+          const uint32_t y = __shfl_up_sync(kFull, incl, o2);
+          if (lane >= o2) incl += y;
+        }
+        uint32_t run = incl - sum;
+#pragma unroll
+        for (int t = 0; t < kPer; ++t) {
+          dbase[kPer * lane + t] = run;
+          run += c[t];
+        }
+      }
+      bar();
+      for (int d = fid; d < kBins; d += NT) {
+        uint32_t run = dbase[d];
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) {
+          const uint32_t t = cnt[ww * kBins + d];
+          cnt[ww * kBins + d] = static_cast<CT>(run);
+          run += t;
+        }
+      }
+      bar();
+      // scatter in order
+      for (int c0 = i0; c0 < i1; c0 += 32) {
+        const int i = c0 + lane;
+        const bool v = i < i1;
+        uint32_t d = 0u, e = 0u;
+        if (v) {
+          e = pa[i];
+          d = ((half ? kmax - s.hkey[e] : s.hidx[e]) >> sh) & (kBins - 1);
+        }
+        uint32_t peers = __ballot_sync(kFull, v);
+#pragma unroll
+        for (int bit = 0; bit < BITS; ++bit) {
+          const uint32_t bb = __ballot_sync(kFull, (d >> bit) & 1u);
+          peers &= ((d >> bit) & 1u) ? bb : ~bb;
+        }
+        const uint32_t base = v ? static_cast<uint32_t>(cnt[fw * kBins + d]) : 0u;
+        if (v) pb[base + __popc(peers & lt)] = static_cast<uint16_t>(e);
+        __syncwarp();
+        if (v && (peers & lt) == 0u) cnt[fw * kBins + d] = static_cast<CT>(base + __popc(peers));
+        __syncwarp();
+      }
+      bar();
+      uint16_t* t = pa;
+      pa = pb;
+      pb = t;
+    }
+  }
+
   // Candidates [0, n) ordered by the composite C = (kmax - key) << 32 | index
   // (key descending, index ascending) with a stable LSD radix sort of a
-  // 16-bit permutation, one counting pass per byte of C that differs between
-  // candidates (values on a coarse grid leave most key bytes equal), then the
-  // first m written. Used when buckets stay crowded with equal keys, where
-  // counting ranks inside a bucket would be quadratic. Ends with a barrier.
+  // 16-bit permutation, then the first m written. Used when buckets stay
+  // crowded with equal keys (values on a coarse grid, such as fp8 or bf16),
+  // where counting ranks inside a bucket would be quadratic. Digits of 8 or 9
+  // bits (whichever needs fewer passes; 8 on a tie) are laid over the span
+  // of bits that differ between candidates in each half of C (the indices of
+  // a 128K row take two 9-bit passes, three 8-bit ones). Ends with a barrier.
   //   per pass: each warp owns a contiguous range of the current order and
   //   walks it 32 at a time; lanes holding the same digit are matched with
-  //   eight ballots; per-warp digit counts are scanned digit-major, warp-minor,
-  //   so the scatter keeps the current order among equal digits.
+  //   one ballot per digit bit; per-warp digit counts are scanned
+  //   digit-major, warp-minor, so the scatter keeps the current order among
+  //   equal digits.
   __device__ __noinline__ static void finish_sorted(Smem& s, int n, int m, int k, uint32_t kmax, int64_t row,
                                                     const Params p, int fid) {
     const int fw = fid >> 5, lane = fid & 31;
     int32_t* o = p.out + row * static_cast<int64_t>(k);
     uint16_t* pa = s.perm;
     uint16_t* pb = reinterpret_cast<uint16_t*>(s.ostage);  // 2 x kMaxK bytes = kHandCap entries
-    uint32_t* cnt = s.bcnt;                                // [kWarps][256] per-warp digit counts
-    uint32_t* dbase = s.bcnt + kWarps * 256;               // [256] digit starts
-    // bytes of C that vary: from the OR and AND of its two halves
+    // bits of C that vary: from the OR and AND of its two halves
     uint32_t or_hi = 0u, and_hi = 0xFFFFFFFFu, or_lo = 0u, and_lo = 0xFFFFFFFFu;
     for (int e = fid; e < n; e += NT) {
       const uint32_t hi = kmax - s.hkey[e], lo = s.hidx[e];
@@ -1063,99 +1172,16 @@ struct Finisher {
       vhi = a0 & ~a1;
       vlo = b0 & ~b1;
     }
-    const int per = ((n + kWarps - 1) / kWarps + 31) & ~31;  // items per warp, whole chunks
-    const int i0 = fw * per, i1 = min(n, i0 + per);
-    const uint32_t lt = lanemask_lt();
-    for (int byte = 0; byte < 8; ++byte) {
-      const uint32_t vary = byte < 4 ? (vlo >> (8 * byte)) & 255u : (vhi >> (8 * (byte - 4))) & 255u;
-      if (vary == 0u) continue;  // the same in every candidate: the pass would be the identity
-      const int sh = 8 * (byte & 3);
-      const bool hi_half = byte >= 4;
-      for (int d = lane; d < 256; d += 32) cnt[fw * 256 + d] = 0u;
-      __syncwarp();
-      // count
-      for (int c0 = i0; c0 < i1; c0 += 32) {
-        const int i = c0 + lane;
-        const bool v = i < i1;
-        uint32_t d = 0u;
-        if (v) {
-          const uint32_t e = pa[i];
-          d = ((hi_half ? kmax - s.hkey[e] : s.hidx[e]) >> sh) & 255u;
-        }
-        uint32_t peers = __ballot_sync(kFull, v);
-#pragma unroll
-        for (int bit = 0; bit < 8; ++bit) {
-          const uint32_t bb = __ballot_sync(kFull, (d >> bit) & 1u);
-          peers &= ((d >> bit) & 1u) ? bb : ~bb;
-        }
-        if (v && (peers & lt) == 0u) cnt[fw * 256 + d] += __popc(peers);
-        __syncwarp();
-      }
-      bar();
-      // digit starts: digit-major, warp-minor exclusive prefix
-      for (int d = fid; d < 256; d += NT) {
-        uint32_t t = 0;
-#pragma unroll
-        for (int ww = 0; ww < kWarps; ++ww) t += cnt[ww * 256 + d];
-        dbase[d] = t;
-      }
-      bar();
-      if (fw == 0) {
-        uint32_t c[8], sum = 0;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          c[t] = dbase[8 * lane + t];
-          sum += c[t];
-        }
-        uint32_t incl = sum;
-#pragma unroll
-        for (int o2 = 1; o2 < 32; o2 <<= 1) {
-          const uint32_t y = __shfl_up_sync(kFull, incl, o2);
-          if (lane >= o2) incl += y;
-        }
-        uint32_t run = incl - sum;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          dbase[8 * lane + t] = run;
-          run += c[t];
-        }
-      }
-      bar();
-      for (int d = fid; d < 256; d += NT) {
-        uint32_t run = dbase[d];
-#pragma unroll
-        for (int ww = 0; ww < kWarps; ++ww) {
-          const uint32_t t = cnt[ww * 256 + d];
-          cnt[ww * 256 + d] = run;
-          run += t;
-        }
-      }
-      bar();
-      // scatter in order
-      for (int c0 = i0; c0 < i1; c0 += 32) {
-        const int i = c0 + lane;
-        const bool v = i < i1;
-        uint32_t d = 0u, e = 0u;
-        if (v) {
-          e = pa[i];
-          d = ((hi_half ? kmax - s.hkey[e] : s.hidx[e]) >> sh) & 255u;
-        }
-        uint32_t peers = __ballot_sync(kFull, v);
-#pragma unroll
-        for (int bit = 0; bit < 8; ++bit) {
-          const uint32_t bb = __ballot_sync(kFull, (d >> bit) & 1u);
-          peers &= ((d >> bit) & 1u) ? bb : ~bb;
-        }
-        const uint32_t base = v ? cnt[fw * 256 + d] : 0u;
-        if (v) pb[base + __popc(peers & lt)] = static_cast<uint16_t>(e);
-        __syncwarp();
-        if (v && (peers & lt) == 0u) cnt[fw * 256 + d] = base + __popc(peers);
-        __syncwarp();
-      }
-      bar();
-      uint16_t* t = pa;
-      pa = pb;
-      pb = t;
+    auto span = [](uint32_t v) { return v ? (31 - __clz(v)) - (__ffs(v) - 1) + 1 : 0; };
+    auto passes = [&](int bits) { return (span(vlo) + bits - 1) / bits + (span(vhi) + bits - 1) / bits; };
+    const bool wide = passes(9) < passes(8);
+    for (int half = 0; half < 2; ++half) {
+      const uint32_t vary = half ? vhi : vlo;
+      if (vary == 0u) continue;  // the same in every candidate: its passes would be the identity
+      if (wide)
+        radix_passes<9>(s, n, kmax, half, vary, pa, pb, fid);
+      else
+        radix_passes<8>(s, n, kmax, half, vary, pa, pb, fid);
     }
     const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
     if (fid == 0) {
@@ -1275,7 +1301,13 @@ struct Finisher {
       bar();
 #pragma unroll
       for (int ww = 0; ww < kWarps; ++ww) big = max(big, s.nred[4][ww]);
-      if (big <= static_cast<uint32_t>(kSmallBucket) || sh == 0 || pass == kSortPasses - 1) break;
+      // a bucket still crowded past the counting limit after a second, finer
+      // pass holds values on a coarse grid (equal keys), which finer slices of
+      // the same composite range do not split: sort instead (the first pass
+      // alone can be coarse when the keys span both signs)
+      if (big <= static_cast<uint32_t>(kSmallBucket) || (pass >= 1 && big > static_cast<uint32_t>(kBigBucket)) ||
+          sh == 0 || pass == kSortPasses - 1)
+        break;
       cmax = ((static_cast<uint64_t>(bm) + 1u) << sh) - 1u;
       sh = bucket_shift(cmax);
       bar();  // bc[4] and nred[4] are rewritten by the next pass
