@@ -821,88 +821,6 @@ __device__ __forceinline__ void stream_item(Smem& s, Filter& f, RingPos& rp, con
   bar_filter();  // every append is visible
 }
 
-template <class T>
-__device__ void filter_loop(Smem& s, const Params& p, int tid) {
-  const int lane = tid & 31;
-  const T* logits = static_cast<const T*>(p.logits);
-  const int k = p.k;
-  RingPos rp{0, 0u, 0u};
-  Filter f;
-  f.par = 0;
-  int h = 0;
-  int64_t row = blockIdx.x;
-  int32_t L_next = row < p.num_rows ? static_cast<int32_t>(clamp_len(p.lengths, row, p.row_stride)) : 0;
-  for (; row < p.num_rows; row += gridDim.x, ++h) {
-    if (s.abort_seen) return;  // a wait gave up during the previous row: the filter warps leave together
-    const int32_t L = L_next;  // lengths are int32, so is every clamped length
-    if (row + gridDim.x < p.num_rows)
-      L_next = static_cast<int32_t>(clamp_len(p.lengths, row + gridDim.x, p.row_stride));
-    const int m = static_cast<int>(min64(k, L));
-    const T* rowp = logits + row * p.row_stride;
-    const RowSpan sp = row_span(rowp, L);
-    const int eb = h & 1;  // estimate written by the finisher two rows back
-    bool spec = false;
-    f.t = __int_as_float(0xff800000);
-    if (m == k) {
-      if (s.est_ok[eb] && L >= s.est_len[eb] - (s.est_len[eb] >> 3)) {
-        spec = true;
-        f.t = s.est[eb];
-      } else if (s.own_len > 0 && L >= s.own_len - (s.own_len >> 3)) {
-        spec = true;
-        f.t = s.own_key > kInfKey ? __int_as_float(0x7f800000) : from_key(s.own_key);
-      }
-    }
-    if (m == k && !spec && L >= kSampleMinLen) {
-      const float ts = sample_threshold(s, rowp, L, m, tid);
-      if (ts > __int_as_float(0xff800000)) {
-        spec = true;
-        f.t = ts;
-      }
-    }
-    if (tid == 0) s.row_t0 = f.t;  // the row's initial threshold (read by thread 0 at the row's end)
-    f.cnt = 0;
-    f.compacted = false;
-    f.strict = false;
-    f.bounded = false;
-    stream_item<T>(s, f, rp, sp, L, 0u, m, tid);
-    const bool reread = spec && !f.compacted && f.cnt < static_cast<uint32_t>(m) && !s.abort_seen;
-    if (reread) {
-      if (tid == 0) atomicOr(&g_status, kStatusReread);
-      f = refilter_from_global<T>(s, f, sp, L, 0u, m, tid);
-    }
-    if (f.cnt > static_cast<uint32_t>(kHandCap)) compact_any(s, f, m, tid);
-    if (tid == 0 && m == k) {
-      // carried to the CTA's next row: a speculative threshold that passed at
-      // least m values of this row (it needed no re-read), else the bound the
-      // filter ended with. A compaction's cut is a poor carry: it can sit
-      // just under this row's m-th value and above a similar row's.
-      if (spec && !reread) {
-        s.own_key = to_key(s.row_t0);
-        s.own_len = L;
-      } else if (f.bounded) {
-        s.own_key = f.last_key;
-        s.own_len = L;
-      }
-    }
-    bar_filter();  // the own estimate is read at the next row's start
-    // hand over: wait until the finishers released the previous handover (a
-    // wait that gave up hands over regardless; the row's output is undefined)
-    mbar_wait_sleep(&s.hempty, (h & 1) ^ 1, &s.wait);
-    for (int e = tid; e < static_cast<int>(f.cnt); e += kFilterThreads) {
-      s.hkey[e] = s.fkey[e];
-      s.hidx[e] = s.fidx[e];
-    }
-    if (tid == 0) {
-      s.h_row = row;
-      s.h_len = L;
-      s.h_n = static_cast<int32_t>(f.cnt);
-      s.h_m = m;
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&s.hfull);
-  }
-}
-
 // ---------------------------------------------------------- finisher
 // Ranks candidates hkey/hidx [0, n) by the composite C = (kmax - key) << 32 |
 // index (ascending C = key descending, index ascending; all C distinct) and
@@ -1385,7 +1303,99 @@ struct Finisher {
 };
 
 using RowFinisher = Finisher<kFinishThreads, 2>;
+// the filter warps' own ranking: a cluster leader's row, and a CTA's last row
 using LeaderFinisher = Finisher<kFilterThreads, 1>;
+
+template <class T>
+__device__ void filter_loop(Smem& s, const Params& p, int tid) {
+  const int lane = tid & 31;
+  const T* logits = static_cast<const T*>(p.logits);
+  const int k = p.k;
+  RingPos rp{0, 0u, 0u};
+  Filter f;
+  f.par = 0;
+  int h = 0;
+  int64_t row = blockIdx.x;
+  int32_t L_next = row < p.num_rows ? static_cast<int32_t>(clamp_len(p.lengths, row, p.row_stride)) : 0;
+  for (; row < p.num_rows; row += gridDim.x, ++h) {
+    if (s.abort_seen) return;  // a wait gave up during the previous row: the filter warps leave together
+    const int32_t L = L_next;  // lengths are int32, so is every clamped length
+    if (row + gridDim.x < p.num_rows)
+      L_next = static_cast<int32_t>(clamp_len(p.lengths, row + gridDim.x, p.row_stride));
+    const int m = static_cast<int>(min64(k, L));
+    const T* rowp = logits + row * p.row_stride;
+    const RowSpan sp = row_span(rowp, L);
+    const int eb = h & 1;  // estimate written by the finisher two rows back
+    bool spec = false;
+    f.t = __int_as_float(0xff800000);
+    if (m == k) {
+      if (s.est_ok[eb] && L >= s.est_len[eb] - (s.est_len[eb] >> 3)) {
+        spec = true;
+        f.t = s.est[eb];
+      } else if (s.own_len > 0 && L >= s.own_len - (s.own_len >> 3)) {
+        spec = true;
+        f.t = s.own_key > kInfKey ? __int_as_float(0x7f800000) : from_key(s.own_key);
+      }
+    }
+    if (m == k && !spec && L >= kSampleMinLen) {
+      const float ts = sample_threshold(s, rowp, L, m, tid);
+      if (ts > __int_as_float(0xff800000)) {
+        spec = true;
+        f.t = ts;
+      }
+    }
+    if (tid == 0) s.row_t0 = f.t;  // the row's initial threshold (read by thread 0 at the row's end)
+    f.cnt = 0;
+    f.compacted = false;
+    f.strict = false;
+    f.bounded = false;
+    stream_item<T>(s, f, rp, sp, L, 0u, m, tid);
+    const bool reread = spec && !f.compacted && f.cnt < static_cast<uint32_t>(m) && !s.abort_seen;
+    if (reread) {
+      if (tid == 0) atomicOr(&g_status, kStatusReread);
+      f = refilter_from_global<T>(s, f, sp, L, 0u, m, tid);
+    }
+    if (f.cnt > static_cast<uint32_t>(kHandCap)) compact_any(s, f, m, tid);
+    if (tid == 0 && m == k) {
+      // carried to the CTA's next row: a speculative threshold that passed at
+      // least m values of this row (it needed no re-read), else the bound the
+      // filter ended with. A compaction's cut is a poor carry: it can sit
+      // just under this row's m-th value and above a similar row's.
+      if (spec && !reread) {
+        s.own_key = to_key(s.row_t0);
+        s.own_len = L;
+      } else if (f.bounded) {
+        s.own_key = f.last_key;
+        s.own_len = L;
+      }
+    }
+    bar_filter();  // the own estimate is read at the next row's start
+    // hand over: wait until the finishers released the previous handover (a
+    // wait that gave up hands over regardless; the row's output is undefined)
+    mbar_wait_sleep(&s.hempty, (h & 1) ^ 1, &s.wait);
+    for (int e = tid; e < static_cast<int>(f.cnt); e += kFilterThreads) {
+      s.hkey[e] = s.fkey[e];
+      s.hidx[e] = s.fidx[e];
+    }
+    if (row + gridDim.x >= p.num_rows) {
+      // the CTA's last row: the finisher warps have stopped after the row
+      // before it, and nothing else is left to stream, so the filter warps
+      // rank it themselves (more threads, no handover latency)
+      bar_filter();  // the copied candidates are visible
+      LeaderFinisher::finish(s, static_cast<int>(f.cnt), m, k, row, p, tid, true);
+      return;
+    }
+    if (tid == 0) {
+      s.h_row = row;
+      s.h_len = L;
+      s.h_n = static_cast<int32_t>(f.cnt);
+      s.h_m = m;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.hfull);
+  }
+}
+
 
 // The estimate the filter starts a later row from: the k-th value minus half
 // the gap to the 3k/4-th, and at least one step of the element type's value
@@ -1404,12 +1414,13 @@ __device__ void finish_loop(Smem& s, const Params& p, int fid) {
   const int lane = fid & 31;
   const int k = p.k;
   int h = 0;
-  for (int64_t row = blockIdx.x; row < p.num_rows; row += gridDim.x, ++h) {
+  // rows up to, not including, the CTA's last: the filter warps rank that one
+  for (int64_t row = blockIdx.x; row + gridDim.x < p.num_rows; row += gridDim.x, ++h) {
     const bool ok = mbar_wait_sleep(&s.hfull, h & 1, &s.wait);
     if (bar_any<2, kFinishThreads>(!ok)) return;  // the filter warps left: nothing more comes
     const int n = s.h_n, m = s.h_m;
     const int64_t L = s.h_len;
-    RowFinisher::finish(s, n, m, k, s.h_row, p, fid, row + gridDim.x >= p.num_rows);
+    RowFinisher::finish(s, n, m, k, s.h_row, p, fid, false);
     if (fid == 0) {
       bool est_ok = false;
       float e = 0.f;
