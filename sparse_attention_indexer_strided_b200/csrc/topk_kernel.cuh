@@ -165,6 +165,14 @@ struct __align__(128) Smem {
   unsigned long long hfull, hempty;
 };
 static_assert(sizeof(Smem) <= 232448, "shared memory budget of one CTA per SM");
+
+// The CTA's shared-memory block. Functions that are not inlined take it from
+// here, not as an argument: through a reference argument every access would
+// be a generic one (slower than a shared-memory access, atomics most of all).
+__device__ __forceinline__ Smem& cta_smem() {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  return *reinterpret_cast<Smem*>(smem_raw);
+}
 static_assert(2 * 256 + 256 <= kBucketMax, "merge histograms alias the bucket counters");
 
 __device__ __forceinline__ void bar_filter() { asm volatile("bar.sync 1, %0;" ::"n"(kFilterThreads) : "memory"); }
@@ -471,7 +479,8 @@ __device__ void count_gt_eq(Smem& s, int n, uint32_t T, uint32_t& ngt, uint32_t&
 
 // Exact: keeps the top m of candidates [0, n) by (key descending, index
 // ascending), n > m >= 1. Returns the m-th largest key.
-__device__ __noinline__ uint32_t compact_exact(Smem& s, int n, int m, int tid) {
+__device__ __noinline__ uint32_t compact_exact(int n, int m, int tid) {
+  Smem& s = cta_smem();
   bar_filter();  // every append is visible
   const uint32_t T = filter_kth(s, n, static_cast<uint32_t>(m), FKey{&s}, FAll{}, tid);
   uint32_t ngt, neq;
@@ -492,7 +501,8 @@ struct FastCut {
   uint32_t ok, lo, kept;
 };
 
-__device__ __noinline__ FastCut compact_fast(Smem& s, int n, int m, int tid) {
+__device__ __noinline__ FastCut compact_fast(int n, int m, int tid) {
+  Smem& s = cta_smem();
   uint32_t kept = 0;
   const int w = tid >> 5, lane = tid & 31;
   bar_filter();  // every append is visible
@@ -556,7 +566,7 @@ __device__ __forceinline__ void tighten(Filter& f, int m) {
 
 // Bounds the buffer again: the approximate pass, else the exact one.
 __device__ __forceinline__ void compact_any(Smem& s, Filter& f, int m, int tid) {
-  const FastCut c = compact_fast(s, static_cast<int>(f.cnt), m, tid);
+  const FastCut c = compact_fast(static_cast<int>(f.cnt), m, tid);
   if (c.ok) {
     f.cnt = c.kept;
     f.t = c.lo > kInfKey ? __int_as_float(0x7f800000) : from_key(c.lo);
@@ -565,7 +575,7 @@ __device__ __forceinline__ void compact_any(Smem& s, Filter& f, int m, int tid) 
     f.strict = false;
     tighten(f, m);
   } else {
-    const uint32_t T = compact_exact(s, static_cast<int>(f.cnt), m, tid);
+    const uint32_t T = compact_exact(static_cast<int>(f.cnt), m, tid);
     f.cnt = static_cast<uint32_t>(m);
     f.t = above(T);
     f.last_key = T;
@@ -736,7 +746,8 @@ __device__ __forceinline__ Filter refilter_from_global(Smem& s, Filter f, RowSpa
 // more in candidate writes and compactions than it saves. Returns -inf when
 // the sample gives none.
 template <class T>
-__device__ __noinline__ float sample_threshold(Smem& s, const T* row, int64_t L, int m, int tid) {
+__device__ __noinline__ float sample_threshold(const T* row, int64_t L, int m, int tid) {
+  Smem& s = cta_smem();
   const int w = tid >> 5, lane = tid & 31;
   const uintptr_t a = reinterpret_cast<uintptr_t>(row);
   const uintptr_t as = a & ~static_cast<uintptr_t>(15);
@@ -931,49 +942,53 @@ struct Finisher {
     }
   }
 
-  // One stable LSD pass per BITS-bit digit over [lo_bit, hi_bit] of one half
-  // of C (half 0: the index, half 1: kmax - key), moving the permutation from
-  // *pa to *pb and swapping them. Counters are 32-bit where they fit beside
-  // the digit starts in the bucket-counter space, else 16-bit (n <= 4096).
-  template <int BITS>
+  // One stable LSD pass per 8-bit digit over [lo_bit, hi_bit] of one half of
+  // C (half 0: the index, half 1: kmax - key), moving the permutation from *pa
+  // to *pb and swapping them. Each warp owns a contiguous range of the
+  // current order. Counting needs no order: every lane adds one to its
+  // warp's counter for its digit (16-bit counters, two to a word). The
+  // scatter walks the warp's chunks of 32 in order; the lanes holding one
+  // digit find one another through a per-warp lane-mask word per digit
+  // (atomicOr, read back, cleared by the group's first lane), and take
+  // consecutive places after that digit's running position. (One vote per
+  // digit bit, or match.any, costs several times more here.) The masks are
+  // zero on entry and on return.
   __device__ __forceinline__ static void radix_passes(Smem& s, int n, uint32_t kmax, int half, uint32_t vary,
                                                       uint16_t*& pa, uint16_t*& pb, int fid) {
-    constexpr int kBins = 1 << BITS;
-    using CT = typename std::conditional<(kWarps + 1) * kBins * 4 <= kBucketMax * 4, uint32_t, uint16_t>::type;
+    constexpr int kBins = 256;
+    static_assert(kWarps * kBins + kWarps * kBins / 2 + kBins <= kBucketMax && kHandCap < 65536,
+                  "lane masks, 16-bit digit counters and digit starts fit the bucket space");
     const int fw = fid >> 5, lane = fid & 31;
-    CT* cnt = reinterpret_cast<CT*>(s.bcnt);  // [kWarps][kBins] per-warp digit counts
-    uint32_t* dbase = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(s.bcnt) + kWarps * kBins * sizeof(CT));
+    uint32_t* mw = s.bcnt + fw * kBins;  // this warp's lane masks
+    uint32_t* cwords = s.bcnt + kWarps * kBins;
+    uint32_t* cw = cwords + fw * (kBins / 2);                 // this warp's counters, as words
+    uint16_t* ch = reinterpret_cast<uint16_t*>(cwords);       // [kWarps][kBins] counters
+    uint16_t* mine = ch + fw * kBins;
+    uint32_t* dbase = cwords + kWarps * (kBins / 2);          // [kBins] digit starts
     const int per = ((n + kWarps - 1) / kWarps + 31) & ~31;  // items per warp, whole chunks
     const int i0 = fw * per, i1 = min(n, i0 + per);
     const uint32_t lt = lanemask_lt();
     const int lo_bit = __ffs(vary) - 1, hi_bit = 31 - __clz(vary);
-    for (int sh = lo_bit; sh <= hi_bit; sh += BITS) {
-      for (int d = lane; d < kBins; d += 32) cnt[fw * kBins + d] = 0;
+    for (int sh = lo_bit; sh <= hi_bit; sh += 8) {
+      auto digit = [&](uint32_t e) -> uint32_t {
+        return ((half ? kmax - s.hkey[e] : s.hidx[e]) >> sh) & (kBins - 1);
+      };
+      for (int d = lane; d < kBins / 2; d += 32) cw[d] = 0u;
       __syncwarp();
-      // count
+#pragma unroll 4
       for (int c0 = i0; c0 < i1; c0 += 32) {
         const int i = c0 + lane;
-        const bool v = i < i1;
-        uint32_t d = 0u;
-        if (v) {
-          const uint32_t e = pa[i];
-          d = ((half ? kmax - s.hkey[e] : s.hidx[e]) >> sh) & (kBins - 1);
+        if (i < i1) {
+          const uint32_t d = digit(pa[i]);
+          atomicAdd(&cw[d >> 1], 1u << (16u * (d & 1u)));
         }
-        uint32_t peers = __ballot_sync(kFull, v);
-#pragma unroll
-        for (int bit = 0; bit < BITS; ++bit) {
-          const uint32_t bb = __ballot_sync(kFull, (d >> bit) & 1u);
-          peers &= ((d >> bit) & 1u) ? bb : ~bb;
-        }
-        if (v && (peers & lt) == 0u) cnt[fw * kBins + d] = static_cast<CT>(cnt[fw * kBins + d] + __popc(peers));
-        __syncwarp();
       }
       bar();
-      // digit starts: digit-major, warp-minor exclusive prefix
+      // digit totals; their exclusive scan (warp 0); each warp's start per digit
       for (int d = fid; d < kBins; d += NT) {
         uint32_t t = 0;
 #pragma unroll
-        for (int ww = 0; ww < kWarps; ++ww) t += cnt[ww * kBins + d];
+        for (int ww = 0; ww < kWarps; ++ww) t += ch[ww * kBins + d];
         dbase[d] = t;
       }
       bar();
@@ -1003,31 +1018,34 @@ struct Finisher {
         uint32_t run = dbase[d];
 #pragma unroll
         for (int ww = 0; ww < kWarps; ++ww) {
-          const uint32_t t = cnt[ww * kBins + d];
-          cnt[ww * kBins + d] = static_cast<CT>(run);
+          const uint32_t t = ch[ww * kBins + d];
+          ch[ww * kBins + d] = static_cast<uint16_t>(run);
           run += t;
         }
       }
       bar();
-      // scatter in order
+      // scatter in order; the next chunk's item and digit are loaded ahead
+      bool vn = i0 + lane < i1;
+      uint32_t en = vn ? pa[i0 + lane] : 0u;
+      uint32_t dn = vn ? digit(en) : 0u;
       for (int c0 = i0; c0 < i1; c0 += 32) {
-        const int i = c0 + lane;
-        const bool v = i < i1;
-        uint32_t d = 0u, e = 0u;
-        if (v) {
-          e = pa[i];
-          d = ((half ? kmax - s.hkey[e] : s.hidx[e]) >> sh) & (kBins - 1);
+        const bool v = vn;
+        const uint32_t e = en, d = dn;
+        vn = c0 + 32 + lane < i1;
+        if (vn) {
+          en = pa[c0 + 32 + lane];
+          dn = digit(en);
         }
-        uint32_t peers = __ballot_sync(kFull, v);
-#pragma unroll
-        for (int bit = 0; bit < BITS; ++bit) {
-          const uint32_t bb = __ballot_sync(kFull, (d >> bit) & 1u);
-          peers &= ((d >> bit) & 1u) ? bb : ~bb;
-        }
-        const uint32_t base = v ? static_cast<uint32_t>(cnt[fw * kBins + d]) : 0u;
+        if (v) atomicOr(&mw[d], 1u << lane);
+        __syncwarp();
+        const uint32_t peers = v ? mw[d] : 0u;
+        const uint32_t base = v ? mine[d] : 0u;
         if (v) pb[base + __popc(peers & lt)] = static_cast<uint16_t>(e);
         __syncwarp();
-        if (v && (peers & lt) == 0u) cnt[fw * kBins + d] = static_cast<CT>(base + __popc(peers));
+        if (v && (peers & lt) == 0u) {
+          mw[d] = 0u;
+          mine[d] = static_cast<uint16_t>(base + __popc(peers));
+        }
         __syncwarp();
       }
       bar();
@@ -1037,34 +1055,49 @@ struct Finisher {
     }
   }
 
-  // Candidates [0, n) ordered by the composite C = (kmax - key) << 32 | index
-  // (key descending, index ascending) with a stable LSD radix sort of a
-  // 16-bit permutation, then the first m written. Used when buckets stay
-  // crowded with equal keys (values on a coarse grid, such as fp8 or bf16),
-  // where counting ranks inside a bucket would be quadratic. Digits of 8 or 9
-  // bits (whichever needs fewer passes; 8 on a tie) are laid over the span
-  // of bits that differ between candidates in each half of C (the indices of
-  // a 128K row take two 9-bit passes, three 8-bit ones). Ends with a barrier.
-  //   per pass: each warp owns a contiguous range of the current order and
-  //   walks it 32 at a time; lanes holding the same digit are matched with
-  //   one ballot per digit bit; per-warp digit counts are scanned
-  //   digit-major, warp-minor, so the scatter keeps the current order among
-  //   equal digits.
-  __device__ __noinline__ static void finish_sorted(Smem& s, int n, int m, int k, uint32_t kmax, int64_t row,
+  // Candidates with C <= cut (every rank below m among them) ordered by the
+  // composite C = (kmax - key) << 32 | index (key descending, index
+  // ascending) with a stable LSD radix sort of a 16-bit permutation, then the
+  // first m written. Used when buckets stay crowded with equal keys (values
+  // on a coarse grid, such as fp8 or bf16), where counting ranks inside a
+  // bucket would be quadratic. The 8-bit digits are laid over the span of
+  // bits that differ between the sorted candidates in each half of C (the
+  // indices of a 64K row take two passes, keys on the fp8 grid one). Ends
+  // with a barrier.
+  __device__ __noinline__ static void finish_sorted(int n, int m, int k, uint32_t kmax, uint64_t cut, int64_t row,
                                                     const Params p, int fid) {
+    Smem& s = cta_smem();
     const int fw = fid >> 5, lane = fid & 31;
     int32_t* o = p.out + row * static_cast<int64_t>(k);
     uint16_t* pa = s.perm;
     uint16_t* pb = reinterpret_cast<uint16_t*>(s.ostage);  // 2 x kMaxK bytes = kHandCap entries
-    // bits of C that vary: from the OR and AND of its two halves
+    for (int i = fid; i < kWarps * 256; i += NT) s.bcnt[i] = 0u;  // the radix passes' lane masks
+    if (fid == 0) s.bc[6] = 0u;
+    bar();
+    // the candidates to sort, and the bits of C that vary among them (from
+    // the OR and AND of its two halves)
     uint32_t or_hi = 0u, and_hi = 0xFFFFFFFFu, or_lo = 0u, and_lo = 0xFFFFFFFFu;
-    for (int e = fid; e < n; e += NT) {
-      const uint32_t hi = kmax - s.hkey[e], lo = s.hidx[e];
-      or_hi |= hi;
-      and_hi &= hi;
-      or_lo |= lo;
-      and_lo &= lo;
-      pa[e] = static_cast<uint16_t>(e);
+    const uint32_t lt = lanemask_lt();
+    for (int e0 = 0; e0 < n; e0 += NT) {  // warp-uniform trip count
+      const int e = e0 + fid;
+      bool keep = false;
+      uint32_t hi = 0u, lo = 0u;
+      if (e < n) {
+        hi = kmax - s.hkey[e];
+        lo = s.hidx[e];
+        keep = ((static_cast<uint64_t>(hi) << 32) | lo) <= cut;
+      }
+      const uint32_t b = __ballot_sync(kFull, keep);
+      uint32_t base = 0u;
+      if (lane == 0 && b) base = atomicAdd(&s.bc[6], static_cast<uint32_t>(__popc(b)));
+      base = __shfl_sync(kFull, base, 0);
+      if (keep) {
+        pa[base + __popc(b & lt)] = static_cast<uint16_t>(e);
+        or_hi |= hi;
+        and_hi &= hi;
+        or_lo |= lo;
+        and_lo &= lo;
+      }
     }
     or_hi = __reduce_or_sync(kFull, or_hi);
     and_hi = __reduce_and_sync(kFull, and_hi);
@@ -1077,6 +1110,7 @@ struct Finisher {
       s.nred[3][fw] = and_lo;
     }
     bar();
+    const int ns = static_cast<int>(s.bc[6]);
     uint32_t vhi = 0u, vlo = 0u;
     {
       uint32_t a0 = 0u, a1 = 0xFFFFFFFFu, b0 = 0u, b1 = 0xFFFFFFFFu;
@@ -1090,16 +1124,10 @@ struct Finisher {
       vhi = a0 & ~a1;
       vlo = b0 & ~b1;
     }
-    auto span = [](uint32_t v) { return v ? (31 - __clz(v)) - (__ffs(v) - 1) + 1 : 0; };
-    auto passes = [&](int bits) { return (span(vlo) + bits - 1) / bits + (span(vhi) + bits - 1) / bits; };
-    const bool wide = passes(9) < passes(8);
     for (int half = 0; half < 2; ++half) {
       const uint32_t vary = half ? vhi : vlo;
       if (vary == 0u) continue;  // the same in every candidate: its passes would be the identity
-      if (wide)
-        radix_passes<9>(s, n, kmax, half, vary, pa, pb, fid);
-      else
-        radix_passes<8>(s, n, kmax, half, vary, pa, pb, fid);
+      radix_passes(s, ns, kmax, half, vary, pa, pb, fid);
     }
     const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
     if (fid == 0) {
@@ -1232,8 +1260,9 @@ struct Finisher {
     }
     if (big > static_cast<uint32_t>(kBigBucket)) {
       // many candidates share a bucket (values on a coarse grid): counting
-      // ranks inside it would be quadratic, so sort everything instead
-      finish_sorted(s, n, m, k, kmax, row, p, fid);
+      // ranks inside it would be quadratic, so sort instead, everything up to
+      // the end of the bucket holding rank m-1
+      finish_sorted(n, m, k, kmax, ((static_cast<uint64_t>(s.bc[4]) + 1u) << sh) - 1u, row, p, fid);
       return;
     }
     for (int e = fid; e < n; e += NT) {
@@ -1338,7 +1367,7 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
       }
     }
     if (m == k && !spec && L >= kSampleMinLen) {
-      const float ts = sample_threshold(s, rowp, L, m, tid);
+      const float ts = sample_threshold(rowp, L, m, tid);
       if (ts > __int_as_float(0xff800000)) {
         spec = true;
         f.t = ts;
@@ -1494,8 +1523,9 @@ __device__ void produce_loop(Smem& s, const Params& p) {
 // of every rank run the merge; at the leader (rank 0) the survivors end in
 // hkey/hidx. Returns the number gathered there. The producer warp mirrors
 // every cluster barrier (s.final_bar tells it how many there are).
-__device__ __noinline__ uint32_t cluster_merge(Smem& s, uint32_t n_r, uint32_t m, bool aborted, uint32_t rank,
+__device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool aborted, uint32_t rank,
                                                uint32_t ncta, int tid) {
+  Smem& s = cta_smem();
   const int w = tid >> 5, lane = tid & 31;
   uint32_t nbar = 0;
   uint32_t* phist = s.bcnt;        // [2][256], per rank, read by the others
@@ -1673,7 +1703,8 @@ __device__ __forceinline__ ClusterItem cluster_item(const Params& p) {
 // streams the chunk into the ring; then every warp of the group mirrors the
 // merge's cluster barriers (s.final_bar tells how many), leaving after the last.
 template <class T>
-__device__ __noinline__ void cluster_mirror(Smem& s, const Params p, int tid) {
+__device__ __noinline__ void cluster_mirror(const Params p, int tid) {
+  Smem& s = cta_smem();
   const int w = tid >> 5, lane = tid & 31;
   const ClusterItem it = cluster_item(p);
   if (it.m == 0) return;  // the same for every CTA of the cluster: no merge, no barrier
@@ -1714,7 +1745,7 @@ __device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid
   f.t = __int_as_float(0xff800000);
   bool spec = false;
   if (Lc >= kSampleMinLen && m_r > 0) {
-    const float ts = sample_threshold(s, rowp + it.c0, Lc, static_cast<int>(m_r), tid);
+    const float ts = sample_threshold(rowp + it.c0, Lc, static_cast<int>(m_r), tid);
     if (ts > __int_as_float(0xff800000)) {
       spec = true;
       f.t = ts;
@@ -1736,7 +1767,7 @@ __device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid
     }
     if (f.cnt > static_cast<uint32_t>(kHandCap)) compact_any(s, f, static_cast<int>(m_r), tid);
   }
-  const uint32_t total = cluster_merge(s, f.cnt, it.m, !ok, it.rank, it.ncta, tid);
+  const uint32_t total = cluster_merge(f.cnt, it.m, !ok, it.rank, it.ncta, tid);
   if (it.rank != 0) return;
   if (s.abort_any) {  // some rank gave up: no valid result for this row
     for (int q = tid; q < k; q += kFilterThreads) p.out[it.row * static_cast<int64_t>(k) + q] = -1;
@@ -1791,7 +1822,7 @@ __global__ void __launch_bounds__(rows::kThreads) topk_kernel(const rows::Params
     if (warp < rows::kFilterWarps)
       rows::cluster_filter<T>(s, p, tid);
     else
-      rows::cluster_mirror<T>(s, p, tid);
+      rows::cluster_mirror<T>(p, tid);
   } else if (warp < rows::kFilterWarps) {
     rows::filter_loop<T>(s, p, tid);
   } else if (warp < rows::kProducerWarp) {
