@@ -737,6 +737,92 @@ __device__ __forceinline__ Filter refilter_from_global(Smem& s, Filter f, RowSpa
   return f;
 }
 
+// The need-th largest of the kSampleVals sampled keys in fkey, to within
+// one bin of a second histogram round (1 <= need <= the number sampled; every
+// sampled key lies in [lo, hi]). Round one counts 4096 bins over a 12-bit
+// slice of [lo, hi] below its highest differing bit and finds, from the top,
+// the bin holding the need-th key; round two does the same inside that bin.
+// The result is the smallest sampled key in the final bin: at least `need`
+// sampled keys are at or above it, and at most the rest of that bin besides
+// (for fp32 logits the second round's bins are a few units in the last place
+// wide; for values on a coarse grid the bin is one value, the exact answer).
+// Counters live in fidx, unused until the item streams. Two plain-atomic
+// passes instead of a radix select's three or four rounds with their
+// barriers.
+__device__ __forceinline__ uint32_t sample_kth(Smem& s, uint32_t need, uint32_t lo, uint32_t hi, int tid) {
+  constexpr int kBins = 4096, kPer = kBins / kFilterThreads;  // 16 bins per thread
+  const int w = tid >> 5, lane = tid & 31;
+  uint32_t* hist = s.fidx;
+  const uint32_t span = hi - lo;
+  if (span == 0u) return lo;
+  const int bits = 32 - __clz(span);
+  int sh = bits > 12 ? bits - 12 : 0;  // (key - lo) >> sh < 4096
+  uint32_t base = lo, top = hi;
+  for (int round = 0; round < 2; ++round) {
+    uint4* h4 = reinterpret_cast<uint4*>(hist + kPer * tid);
+#pragma unroll
+    for (int i = 0; i < kPer / 4; ++i) h4[i] = make_uint4(0u, 0u, 0u, 0u);
+    bar_filter();
+    for (int e = tid; e < kSampleVals; e += kFilterThreads) {
+      const uint32_t x = s.fkey[e];
+      if (x >= base && x <= top) atomicAdd(&hist[(x - base) >> sh], 1u);
+    }
+    bar_filter();
+    // from the top: thread tid owns bins kBins - 1 - (kPer tid + j), j = 0..kPer-1
+    const uint4* r4 = reinterpret_cast<const uint4*>(hist + kBins - kPer * (tid + 1));
+    uint32_t c[kPer], sum = 0u;
+#pragma unroll
+    for (int i = 0; i < kPer / 4; ++i) {
+      const uint4 q = r4[i];  // bins ascending; c[] descending
+      c[kPer - 1 - 4 * i] = q.x;
+      c[kPer - 2 - 4 * i] = q.y;
+      c[kPer - 3 - 4 * i] = q.z;
+      c[kPer - 4 - 4 * i] = q.w;
+      sum += q.x + q.y + q.z + q.w;
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t t = __shfl_up_sync(kFull, incl, d);
+      if (lane >= d) incl += t;
+    }
+    if (lane == 31) s.fred[2][w] = incl;
+    bar_filter();
+    uint32_t run = incl - sum;
+    for (int ww = 0; ww < w; ++ww) run += s.fred[2][ww];
+    if (run < need && need <= run + sum) {  // exactly one thread
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        if (run < need && need <= run + c[j]) {
+          s.bc[0] = static_cast<uint32_t>(kBins - 1 - (kPer * tid + j));
+          s.bc[1] = run;
+        }
+        run += c[j];
+      }
+    }
+    bar_filter();
+    const uint32_t b = s.bc[0];
+    need -= s.bc[1];
+    base += b << sh;
+    top = min(top, base + ((1u << sh) - 1u));
+    if (round == 1 || sh == 0) break;
+    sh = sh > 12 ? sh - 12 : 0;
+    bar_filter();  // bc and the counters are rewritten by the next round
+  }
+  // the smallest sampled key in the final bin: a key that occurs (a value
+  // grid's level, so that the filter's strict bound can later exclude its
+  // further copies), with as many keys at or above it as the bin's edge
+  uint32_t mn = 0xFFFFFFFFu;
+  for (int e = tid; e < kSampleVals; e += kFilterThreads) {
+    const uint32_t x = s.fkey[e];
+    if (x >= base && x <= top) mn = min(mn, x);
+  }
+  mn = __reduce_min_sync(kFull, mn);
+  if (lane == 0) s.fred[3][w] = mn;
+  bar_filter();
+  return __reduce_min_sync(kFull, lane < kFilterWarps ? s.fred[3][lane] : 0xFFFFFFFFu);
+}
+
 // A threshold for an item with no estimate, from a sample of kSampleVals
 // values in kSampleChunks evenly spaced runs of 128 (aligned 16-byte blocks
 // inside the item): the value with as many sampled values above it as 1.25
@@ -753,6 +839,7 @@ __device__ __noinline__ float sample_threshold(const T* row, int64_t L, int m, i
   const uintptr_t as = a & ~static_cast<uintptr_t>(15);
   const int64_t j0 = -static_cast<int64_t>((a - as) / sizeof(T));  // item index of the aligned base
   const int64_t span = L - j0;                                      // elements from the aligned base to the end
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
 #pragma unroll
   for (int q = 0; q < kSampleRunsPerWarp; ++q) {
     const int64_t c = w * kSampleRunsPerWarp + q;
@@ -762,13 +849,25 @@ __device__ __noinline__ float sample_threshold(const T* row, int64_t L, int m, i
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int64_t j = j0 + b + 4 * lane + i;
-      s.fkey[c * 128 + lane * 4 + i] = (j >= 0 && j < L) ? to_key(xv[i]) : 0u;  // 0: below every key
+      const uint32_t key = (j >= 0 && j < L) ? to_key(xv[i]) : 0u;  // 0: below every key
+      s.fkey[c * 128 + lane * 4 + i] = key;
+      mn = min(mn, key);
+      mx = max(mx, key);
     }
   }
+  mn = __reduce_min_sync(kFull, mn);
+  mx = __reduce_max_sync(kFull, mx);
+  if (lane == 0) {
+    s.fred[0][w] = mn;
+    s.fred[1][w] = mx;
+  }
   bar_filter();
+  mn = __reduce_min_sync(kFull, lane < kFilterWarps ? s.fred[0][lane] : 0xFFFFFFFFu);
+  mx = __reduce_max_sync(kFull, lane < kFilterWarps ? s.fred[1][lane] : 0u);
   const double share = static_cast<double>(kSampleVals) * m / static_cast<double>(L);
   const uint32_t need = min(static_cast<uint32_t>(kSampleVals - 8), static_cast<uint32_t>(1.25 * share) + 12u);
-  const uint32_t T0 = filter_kth(s, kSampleVals, need, FKey{&s}, FAll{}, tid);
+  const uint32_t T0 = sample_kth(s, need, mn, mx, tid);
+  bar_filter();  // fkey, fidx, fred and bc are free again
   return (T0 == 0u || T0 >= kInfKey) ? __int_as_float(0xff800000) : from_key(T0);
 }
 
