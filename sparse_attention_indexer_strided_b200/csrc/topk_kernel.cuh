@@ -96,7 +96,7 @@ constexpr int kKeepLimit = 2560;                        // approximate compactio
 constexpr int kSampleRunsPerWarp = 4;                   // runs of 128 each filter warp samples
 constexpr int kSampleChunks = kFilterWarps * kSampleRunsPerWarp;  // runs sampled for a row's first threshold
 constexpr int kSampleVals = kSampleChunks * 128;        // 4096 sampled values
-constexpr int64_t kSampleMinLen = 4 * kStageElems;      // shorter rows start with no threshold
+constexpr int64_t kSampleMinLen = 2 * kSampleVals;      // shorter rows start with no threshold
 constexpr int kBigBucket = 64;                          // finisher: larger buckets are sorted instead
 constexpr int kSmallBucket = 16;                        // finisher: largest bucket ranked by direct counting
 constexpr int kSortPasses = 3;                          // finisher: bucket count passes, at most
@@ -288,23 +288,17 @@ __device__ void filter_minmax(Smem& s, int n, V v, P pred, uint32_t& lo, uint32_
 
 // 256-bin histogram of the 8-bit digit at bit sh of v(e), over the entries
 // [0, n) with pred(e) and v(e) in [lo, hi] (hist zeroed, filter threads).
-// Lanes of a warp holding the same digit are merged first (match.any), so
-// one atomic per distinct digit and warp: values on a few levels (ties, the
-// top byte of floats of one sign) would otherwise queue thousands of atomics
-// on one counter.
+// One shared atomic per entry: merging the lanes of a digit first (match.any
+// or a vote per digit bit) costs more than the contended atomics it saves,
+// even for values on a few levels.
 template <class V, class P>
 __device__ __forceinline__ void digit_histogram(uint32_t* hist, int n, V v, P pred, uint32_t lo, uint32_t hi, int sh,
                                                 int tid) {
-  const uint32_t lt = lanemask_lt();
-  for (int e0 = 0; e0 < n; e0 += kFilterThreads) {  // warp-uniform trip count
-    const int e = e0 + tid;
-    uint32_t d = 0xFFFFFFFFu;
-    if (e < n && pred(e)) {
-      const uint32_t x = v(e);
-      if (x >= lo && x <= hi) d = (x >> sh) & 255u;
-    }
-    const uint32_t peers = __match_any_sync(kFull, d);
-    if (d != 0xFFFFFFFFu && (peers & lt) == 0u) atomicAdd(&hist[d], __popc(peers));
+#pragma unroll 4
+  for (int e = tid; e < n; e += kFilterThreads) {
+    if (!pred(e)) continue;
+    const uint32_t x = v(e);
+    if (x >= lo && x <= hi) atomicAdd(&hist[(x >> sh) & 255u], 1u);
   }
 }
 
