@@ -107,13 +107,16 @@ static int device_setup(int dev, DeviceInfo* out) {
 }
 
 // Launch plan from host-known sizes only. A cluster per row pays off when rows
-// are fewer than SMs and long: each rank then streams a chunk of at least
-// kMinChunk elements. The largest cluster size whose whole grid is resident
-// at once is taken (the merge waits on every rank of a cluster).
+// are few and long: each rank then streams a chunk of at least kMinChunk
+// elements. From 32 rows on, one CTA per row finishes sooner unless the rows
+// are long (kLongRow elements and up): the merge costs more than the split
+// saves. The largest cluster size whose whole grid is resident at once is
+// taken (the merge waits on every rank of a cluster).
 static void plan(const DeviceInfo& d, int64_t num_rows, int64_t row_stride, int* cs_out, int64_t* grid_out) {
   constexpr int64_t kMinChunk = 16384;
+  constexpr int64_t kLongRow = 262144;
   int cs = 1;
-  if (num_rows > 0 && num_rows < d.sms) {
+  if (num_rows > 0 && num_rows < d.sms && (num_rows < 32 || row_stride >= kLongRow)) {
     for (int i = 1; i < 5; ++i) {
       const int c = 1 << i;
       if (d.cluster_ctas[i] >= num_rows * c && row_stride / c >= kMinChunk) cs = c;

@@ -1035,9 +1035,9 @@ struct Finisher {
     }
   }
 
-  // One stable LSD pass per 8-bit digit over [lo_bit, hi_bit] of one half of
-  // C (half 0: the index, half 1: kmax - key), moving the permutation from *pa
-  // to *pb and swapping them. Each warp owns a contiguous range of the
+  // One stable LSD pass per digit of up to eight of the bits `vary` of one
+  // half of C (half 0: the index, half 1: kmax - key), lowest bits first,
+  // moving the permutation from *pa to *pb and swapping them. Each warp owns a contiguous range of the
   // current order. Counting needs no order: every lane adds one to its
   // warp's counter for its digit (16-bit counters, two to a word). The
   // scatter walks the warp's chunks of 32 in order; the lanes holding one
@@ -1061,10 +1061,32 @@ struct Finisher {
     const int per = ((n + kWarps - 1) / kWarps + 31) & ~31;  // items per warp, whole chunks
     const int i0 = fw * per, i1 = min(n, i0 + per);
     const uint32_t lt = lanemask_lt();
-    const int lo_bit = __ffs(vary) - 1, hi_bit = 31 - __clz(vary);
-    for (int sh = lo_bit; sh <= hi_bit; sh += 8) {
+    uint32_t rest = vary;
+    while (rest != 0u) {
+      // this pass's digit: the next eight (or fewer) bits that vary, lowest
+      // first; bits that are the same in every candidate do not order them
+      uint32_t dm = 0u;
+      int pos[8], nb = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        pos[i] = 0;
+        if (rest != 0u) {
+          pos[i] = __ffs(rest) - 1;
+          dm |= 1u << pos[i];
+          rest &= rest - 1u;
+          ++nb;
+        }
+      }
+      const int p0 = pos[0];
+      const bool run = ((dm >> p0) & ((dm >> p0) + 1u)) == 0u;  // the bits are contiguous
       auto digit = [&](uint32_t e) -> uint32_t {
-        return ((half ? kmax - s.hkey[e] : s.hidx[e]) >> sh) & (kBins - 1);
+        const uint32_t x = half ? kmax - s.hkey[e] : s.hidx[e];
+        if (run) return (x >> p0) & (dm >> p0);
+        uint32_t d = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (i < nb) d |= ((x >> pos[i]) & 1u) << i;
+        return d;
       };
       for (int d = lane; d < kBins / 2; d += 32) cw[d] = 0u;
       __syncwarp();
@@ -1248,20 +1270,24 @@ struct Finisher {
     int32_t* o = p.out + row * static_cast<int64_t>(k);
     for (int q = m + fid; q < k; q += NT) o[q] = -1;
     if (n <= 0) return;
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, imax = 0u;
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, imax = 0u, kdiff = 0u;
+    const uint32_t key0 = s.hkey[0];
     for (int e = fid; e < n; e += NT) {
       const uint32_t key = s.hkey[e];
       kmin = min(kmin, key);
       kmax = max(kmax, key);
+      kdiff |= key ^ key0;
       imax = max(imax, s.hidx[e]);
     }
     kmin = __reduce_min_sync(kFull, kmin);
     kmax = __reduce_max_sync(kFull, kmax);
     imax = __reduce_max_sync(kFull, imax);
+    kdiff = __reduce_or_sync(kFull, kdiff);
     if (lane == 0) {
       s.nred[0][fw] = kmin;
       s.nred[1][fw] = kmax;
       s.nred[2][fw] = imax;
+      s.nred[3][fw] = kdiff;
     }
     bar();
 #pragma unroll
@@ -1269,7 +1295,12 @@ struct Finisher {
       kmin = min(kmin, s.nred[0][ww]);
       kmax = max(kmax, s.nred[1][ww]);
       imax = max(imax, s.nred[2][ww]);
+      kdiff |= s.nred[3][ww];
     }
+    // every two keys differ by a multiple of 2^grid (keys on a value grid,
+    // such as fp8 or bf16 values, have zero low bits): buckets no wider than
+    // that hold one key each, and finer passes cannot split them
+    const int grid = kdiff ? __ffs(kdiff) - 1 : 32;
     uint64_t cmax = (static_cast<uint64_t>(kmax - kmin) << 32) | imax;
     int sh = bucket_shift(cmax);
     auto comp = [&](uint32_t key, uint32_t idx) -> uint64_t {
@@ -1344,8 +1375,9 @@ struct Finisher {
       // pass holds values on a coarse grid (equal keys), which finer slices of
       // the same composite range do not split: sort instead (the first pass
       // alone can be coarse when the keys span both signs)
-      if (big <= static_cast<uint32_t>(kSmallBucket) || (pass >= 1 && big > static_cast<uint32_t>(kBigBucket)) ||
-          sh == 0 || pass == kSortPasses - 1)
+      if (big <= static_cast<uint32_t>(kSmallBucket) ||
+          (big > static_cast<uint32_t>(kBigBucket) && (pass >= 1 || sh <= 32 + grid)) || sh == 0 ||
+          pass == kSortPasses - 1)
         break;
       cmax = ((static_cast<uint64_t>(bm) + 1u) << sh) - 1u;
       sh = bucket_shift(cmax);

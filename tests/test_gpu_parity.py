@@ -88,7 +88,8 @@ def test_plan_choices(dsa):
     assert dsa.plan(256, 131328, 2048)[0] == 1
     assert dsa.plan(4, 4096, 512)[0] == 1
     assert dsa.plan(4, 900096, 1024)[0] > 1
-    assert dsa.plan(64, 65536, 2048)[0] > 1
+    assert dsa.plan(64, 65536, 2048)[0] == 1  # decode rows: one CTA each
+    assert dsa.plan(64, 300000, 2048)[0] > 1  # many long rows: clusters
 
 
 # ------------------------------------------------------------------ k sweep
@@ -116,6 +117,19 @@ def test_k_sweep_cluster_path(oracle_mod, dsa, k):
     x[2] = np.round(x[2] * 2) / 2
     assert dsa.plan(len(L), stride, k)[0] > 1
     assert_parity(oracle_mod, dsa, x, L, k)
+
+
+def test_cluster_path_many_rows(oracle_mod, dsa):
+    """32 rows and more take clusters only when rows are long: 40 long rows
+    of mixed lengths, every fifth on a coarse grid."""
+    rng = np.random.default_rng(2500)
+    stride = 270000
+    L = rng.integers(0, stride + 1, size=40).astype(np.int32)
+    L[:4] = [stride, 0, 2048, 20000]
+    x = rng.standard_normal((len(L), stride)).astype(np.float32)
+    x[::5] = np.round(x[::5] * 8) / 8
+    assert dsa.plan(len(L), stride, 2048)[0] > 1
+    assert_parity(oracle_mod, dsa, x, L, 2048)
 
 
 # --------------------------------------------------------- layout and poison
