@@ -42,13 +42,22 @@ static std::mutex g_dev_mu;
 template <class T>
 static bool set_kernel_attributes() {
   const int smem = static_cast<int>(sizeof(rows::Smem));
-  if (cudaFuncSetAttribute(topk_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+  if (cudaFuncSetAttribute(topk_rows_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      cudaFuncSetAttribute(topk_cluster_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
-  if (cudaFuncSetAttribute(topk_kernel<T>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+  if (cudaFuncSetAttribute(topk_cluster_kernel<T>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
     cudaGetLastError();  // then only portable sizes (<= 8) launch
   return true;
+}
+
+// The register split needs exactly rows::kLaunchRegs registers per thread.
+template <class T>
+static bool built_with_launch_regs() {
+  cudaFuncAttributes a;
+  return cudaFuncGetAttributes(&a, topk_rows_kernel<T>) == cudaSuccess && a.numRegs == rows::kLaunchRegs &&
+         cudaFuncGetAttributes(&a, topk_cluster_kernel<T>) == cudaSuccess && a.numRegs == rows::kLaunchRegs;
 }
 
 static int device_setup(int dev, DeviceInfo* out) {
@@ -63,17 +72,14 @@ static int device_setup(int dev, DeviceInfo* out) {
     // the library carries sm_100a code only, which runs on compute capability
     // 10.0 alone; the attribute query fails when no image loads on this device
     cudaFuncAttributes fa;
-    if (p.major != 10 || p.minor != 0 || cudaFuncGetAttributes(&fa, topk_kernel<float>) != cudaSuccess) {
+    if (p.major != 10 || p.minor != 0 || cudaFuncGetAttributes(&fa, topk_rows_kernel<float>) != cudaSuccess) {
       cudaGetLastError();
       return DSA_ERR_NO_DEVICE;
     }
     d.sms = p.multiProcessorCount;
     {
-      cudaFuncAttributes a;
-      const bool ok = cudaFuncGetAttributes(&a, topk_kernel<float>) == cudaSuccess && a.numRegs == rows::kLaunchRegs &&
-                      cudaFuncGetAttributes(&a, topk_kernel<__nv_bfloat16>) == cudaSuccess &&
-                      a.numRegs == rows::kLaunchRegs && cudaFuncGetAttributes(&a, topk_kernel<__half>) == cudaSuccess &&
-                      a.numRegs == rows::kLaunchRegs;
+      const bool ok = built_with_launch_regs<float>() && built_with_launch_regs<__nv_bfloat16>() &&
+                      built_with_launch_regs<__half>();
       cudaGetLastError();
       d.regsplit = ok ? 1u : 0u;
     }
@@ -95,7 +101,7 @@ static int device_setup(int dev, DeviceInfo* out) {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int nclusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&nclusters, topk_kernel<float>, &cfg) == cudaSuccess)
+      if (cudaOccupancyMaxActiveClusters(&nclusters, topk_cluster_kernel<float>, &cfg) == cudaSuccess)
         d.cluster_ctas[i] = nclusters * cs;
       else
         cudaGetLastError();
@@ -170,8 +176,8 @@ static int current_device(DeviceInfo* info) {
 }
 
 template <class T>
-static cudaError_t launch_as(const cudaLaunchConfig_t& cfg, const rows::Params& p) {
-  return cudaLaunchKernelEx(&cfg, topk_kernel<T>, p);
+static cudaError_t launch_as(const cudaLaunchConfig_t& cfg, const rows::Params& p, bool clustered) {
+  return clustered ? cudaLaunchKernelEx(&cfg, topk_cluster_kernel<T>, p) : cudaLaunchKernelEx(&cfg, topk_rows_kernel<T>, p);
 }
 
 static int launch(const DeviceInfo& d, int32_t dtype, const rows::Params& p, cudaStream_t stream) {
@@ -198,9 +204,9 @@ static int launch(const DeviceInfo& d, int32_t dtype, const rows::Params& p, cud
   cfg.numAttrs = cs == 1 ? 1 : 2;
   cudaError_t e;
   switch (dtype) {
-    case DSA_DTYPE_F32: e = launch_as<float>(cfg, p); break;
-    case DSA_DTYPE_BF16: e = launch_as<__nv_bfloat16>(cfg, p); break;
-    default: e = launch_as<__half>(cfg, p); break;
+    case DSA_DTYPE_F32: e = launch_as<float>(cfg, p, cs > 1); break;
+    case DSA_DTYPE_BF16: e = launch_as<__nv_bfloat16>(cfg, p, cs > 1); break;
+    default: e = launch_as<__half>(cfg, p, cs > 1); break;
   }
   if (e != cudaSuccess) {
     cudaGetLastError();

@@ -65,6 +65,7 @@ constexpr int kFilterWarps = 8;
 constexpr int kFilterThreads = kFilterWarps * 32;  // 256
 constexpr int kFinishWarps = 6;
 constexpr int kFinishThreads = kFinishWarps * 32;  // 192
+constexpr int kJointThreads = kFilterThreads + kFinishThreads;  // 448: both ranking a CTA's last row
 constexpr int kProducerWarp = kFilterWarps + kFinishWarps;
 constexpr int kThreads = 16 * 32;                       // 512: many-row mode (4 warpgroups; warp 15 idle)
 constexpr int kClusterWarp = kFilterWarps;              // cluster mode: the producer warp
@@ -140,7 +141,7 @@ struct __align__(128) Smem {
   uint32_t hist[256];         // filter radix histogram
   uint4 red[2][(kFilterWarps + 3) / 4];  // per-warp survivor counts, by stage parity
   uint32_t fred[4][kFilterWarps];
-  uint32_t nred[5][kFilterWarps];  // finisher per-warp reductions (6 or 8 warps)
+  uint32_t nred[5][kFilterWarps + kFinishWarps];  // finisher per-warp reductions (6, 8 or 14 warps)
   uint32_t bc[8];
   uint32_t small[32];
   uint32_t rec[2];  // finisher: keys at ranks k-1 and 3k/4-1
@@ -161,6 +162,7 @@ struct __align__(128) Smem {
   uint32_t abort_seen; // the abort flag as thread 0 read it before an item's last filter barrier
   uint32_t abort_any;  // cluster mode: some rank gave up (read by the leader)
   uint32_t final_bar;  // cluster mode: number of cluster barriers of the merge (0: not yet known)
+  uint32_t joint;      // many-row mode: the CTA's last row is ranked by filter and finisher warps together
   unsigned long long full[kMaxStages], empty[kMaxStages];
   unsigned long long hfull, hempty;
 };
@@ -940,9 +942,10 @@ __device__ __forceinline__ void stream_item(Smem& s, Filter& f, RingPos& rp, con
 template <int NT, int BAR>
 struct Finisher {
   static constexpr int kWarps = NT / 32;
-  static constexpr int kBuckets = NT == 192 ? 3840 : 4096;
+  static constexpr int kBuckets = kBucketMax / (4 * NT) * (4 * NT);  // 3840, 4096 or 3584
   static constexpr int kScanPer = kBuckets / NT;  // counters per thread
-  static_assert(kBuckets <= kBucketMax && kBuckets >= 2048 && kScanPer % 4 == 0 && kWarps <= kFilterWarps,
+  static_assert(kBuckets <= kBucketMax && kBuckets >= 2048 && kScanPer % 4 == 0 &&
+                    kWarps <= kFilterWarps + kFinishWarps,
                 "bucket counters split evenly over the threads; bucket_shift narrows a slice by one bit at most");
 
   __device__ __forceinline__ static void bar() { asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory"); }
@@ -1046,14 +1049,19 @@ struct Finisher {
   // consecutive places after that digit's running position. (One vote per
   // digit bit, or match.any, costs several times more here.) The masks are
   // zero on entry and on return.
+  // Scratch of the sort passes: the bucket counters, or with more than eight
+  // warps the filter's candidate buffer (free once the candidates sit in hkey).
+  __device__ __forceinline__ static uint32_t* sort_scratch(Smem& s) { return kWarps > kFilterWarps ? s.fkey : s.bcnt; }
   __device__ __forceinline__ static void radix_passes(Smem& s, int n, uint32_t kmax, int half, uint32_t vary,
                                                       uint16_t*& pa, uint16_t*& pb, int fid) {
     constexpr int kBins = 256;
-    static_assert(kWarps * kBins + kWarps * kBins / 2 + kBins <= kBucketMax && kHandCap < 65536,
-                  "lane masks, 16-bit digit counters and digit starts fit the bucket space");
+    static_assert(kWarps * kBins + kWarps * kBins / 2 + kBins <= (kWarps > kFilterWarps ? kFiltCap : kBucketMax) &&
+                      kHandCap < 65536,
+                  "lane masks, 16-bit digit counters and digit starts fit the sort scratch");
     const int fw = fid >> 5, lane = fid & 31;
-    uint32_t* mw = s.bcnt + fw * kBins;  // this warp's lane masks
-    uint32_t* cwords = s.bcnt + kWarps * kBins;
+    uint32_t* scr = sort_scratch(s);
+    uint32_t* mw = scr + fw * kBins;  // this warp's lane masks
+    uint32_t* cwords = scr + kWarps * kBins;
     uint32_t* cw = cwords + fw * (kBins / 2);                 // this warp's counters, as words
     uint16_t* ch = reinterpret_cast<uint16_t*>(cwords);       // [kWarps][kBins] counters
     uint16_t* mine = ch + fw * kBins;
@@ -1186,7 +1194,8 @@ struct Finisher {
     int32_t* o = p.out + row * static_cast<int64_t>(k);
     uint16_t* pa = s.perm;
     uint16_t* pb = reinterpret_cast<uint16_t*>(s.ostage);  // 2 x kMaxK bytes = kHandCap entries
-    for (int i = fid; i < kWarps * 256; i += NT) s.bcnt[i] = 0u;  // the radix passes' lane masks
+    uint32_t* scr = sort_scratch(s);
+    for (int i = fid; i < kWarps * 256; i += NT) scr[i] = 0u;  // the radix passes' lane masks
     if (fid == 0) s.bc[6] = 0u;
     bar();
     // the candidates to sort, and the bits of C that vary among them (from
@@ -1457,8 +1466,27 @@ struct Finisher {
 };
 
 using RowFinisher = Finisher<kFinishThreads, 2>;
-// the filter warps' own ranking: a cluster leader's row, and a CTA's last row
+// the filter warps' own ranking of a cluster leader's row
 using LeaderFinisher = Finisher<kFilterThreads, 1>;
+// a CTA's last row, ranked by the filter and finisher warps together
+using JointFinisher = Finisher<kJointThreads, 3>;
+
+// Where the filter and finisher warps meet after their row loops. Both roles reach it on every path (a wait that gave up ends a
+// loop early; no loop ends without passing here), so the hardware barrier
+// always completes, and the flag the filter warps wrote before it (s.joint)
+// decides for both whether they rank the row together.
+__device__ __forceinline__ void joint_rendezvous() {
+  asm volatile("bar.sync 3, %0;" ::"n"(kJointThreads) : "memory");
+}
+
+// The joint ranking, out of line (inlined into the row loops, its registers
+// would be allocated with theirs).
+__device__ __noinline__ void joint_finish(const Params p, int tid) {
+  Smem& s = cta_smem();
+  JointFinisher::finish(s, s.h_n, s.h_m, p.k, s.h_row, p, tid, true);
+}
+
+
 
 template <class T>
 __device__ void filter_loop(Smem& s, const Params& p, int tid) {
@@ -1472,7 +1500,7 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
   int64_t row = blockIdx.x;
   int32_t L_next = row < p.num_rows ? static_cast<int32_t>(clamp_len(p.lengths, row, p.row_stride)) : 0;
   for (; row < p.num_rows; row += gridDim.x, ++h) {
-    if (s.abort_seen) return;  // a wait gave up during the previous row: the filter warps leave together
+    if (s.abort_seen) break;  // a wait gave up during the previous row: the filter warps leave together
     const int32_t L = L_next;  // lengths are int32, so is every clamped length
     if (row + gridDim.x < p.num_rows)
       L_next = static_cast<int32_t>(clamp_len(p.lengths, row + gridDim.x, p.row_stride));
@@ -1533,11 +1561,16 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
     }
     if (row + gridDim.x >= p.num_rows) {
       // the CTA's last row: the finisher warps have stopped after the row
-      // before it, and nothing else is left to stream, so the filter warps
-      // rank it themselves (more threads, no handover latency)
-      bar_filter();  // the copied candidates are visible
-      LeaderFinisher::finish(s, static_cast<int>(f.cnt), m, k, row, p, tid, true);
-      return;
+      // before it, and nothing else is left to stream. The only row: both
+      // roles rank it after the rendezvous. Else the filter warps rank it
+      // (no handover latency, in parallel with the finisher warps' last row).
+      if (tid == 0) {
+        s.h_row = row;
+        s.h_n = static_cast<int32_t>(f.cnt);
+        s.h_m = m;
+        s.joint = 1u;
+      }
+      break;
     }
     if (tid == 0) {
       s.h_row = row;
@@ -1548,6 +1581,8 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.hfull);
   }
+  joint_rendezvous();
+  if (s.joint) joint_finish(p, tid);
 }
 
 
@@ -1568,10 +1603,11 @@ __device__ void finish_loop(Smem& s, const Params& p, int fid) {
   const int lane = fid & 31;
   const int k = p.k;
   int h = 0;
-  // rows up to, not including, the CTA's last: the filter warps rank that one
+  // rows up to, not including, the CTA's last (which the filter warps rank,
+  // alone or with these warps)
   for (int64_t row = blockIdx.x; row + gridDim.x < p.num_rows; row += gridDim.x, ++h) {
     const bool ok = mbar_wait_sleep(&s.hfull, h & 1, &s.wait);
-    if (bar_any<2, kFinishThreads>(!ok)) return;  // the filter warps left: nothing more comes
+    if (bar_any<2, kFinishThreads>(!ok)) break;  // the filter warps left: nothing more comes
     const int n = s.h_n, m = s.h_m;
     const int64_t L = s.h_len;
     RowFinisher::finish(s, n, m, k, s.h_row, p, fid, false);
@@ -1592,6 +1628,8 @@ __device__ void finish_loop(Smem& s, const Params& p, int fid) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.hempty);
   }
+  joint_rendezvous();
+  if (s.joint) joint_finish(p, kFilterThreads + fid);
 }
 
 // ---------------------------------------------------------- producer
@@ -1901,60 +1939,77 @@ __device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid
   LeaderFinisher::finish(s, static_cast<int>(total), static_cast<int>(it.m), k, it.row, p, tid, true);
 }
 
+// Shared state of a fresh CTA (thread 0; a barrier follows).
+__device__ __forceinline__ void init_cta(Smem& s) {
+  for (int i = 0; i < kMaxStages; ++i) {
+    mbar_init(&s.full[i], 1);
+    mbar_init(&s.empty[i], kFilterWarps);
+  }
+  mbar_init(&s.hfull, kFilterWarps);
+  mbar_init(&s.hempty, kFinishWarps);
+  for (int i = 0; i < 2; ++i) {
+    s.est_ok[i] = 0;
+    s.est[i] = 0.f;
+    s.est_len[i] = 0;
+  }
+  s.own_key = 0u;
+  s.own_len = 0;
+  s.wait.abort = 0u;
+  s.abort_seen = 0u;
+  s.wait.limit_ns = g_wait_limit_ns;
+  s.abort_any = 0u;
+  s.final_bar = 0u;
+  s.joint = 0u;
+  fence_mbar_init();
+}
+
 }  // namespace rows
 
-// Many rows (cluster size 1): grid = min(num_rows, SMs), one CTA per SM,
-// rows strided by the grid, 512 threads. A cluster per row: grid = num_rows *
-// cluster size, 384 threads.
+// Many rows: grid = min(num_rows, SMs), one CTA per SM, rows strided by the
+// grid, 512 threads. (A kernel of its own, apart from the cluster mode, so
+// that each gets its own register allocation.)
 template <class T>
-__global__ void __launch_bounds__(rows::kThreads) topk_kernel(const rows::Params p) {
+__global__ void __launch_bounds__(rows::kThreads) topk_rows_kernel(const rows::Params p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   rows::Smem& s = *reinterpret_cast<rows::Smem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool clustered = cluster_size() > 1;
-  if (tid == 0) {
-    for (int i = 0; i < rows::kMaxStages; ++i) {
-      mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], rows::kFilterWarps);
-    }
-    mbar_init(&s.hfull, rows::kFilterWarps);
-    mbar_init(&s.hempty, rows::kFinishWarps);
-    for (int i = 0; i < 2; ++i) {
-      s.est_ok[i] = 0;
-      s.est[i] = 0.f;
-      s.est_len[i] = 0;
-    }
-    s.own_key = 0u;
-    s.own_len = 0;
-    s.wait.abort = 0u;
-    s.abort_seen = 0u;
-    s.wait.limit_ns = g_wait_limit_ns;
-    s.abort_any = 0u;
-    s.final_bar = 0u;
-    fence_mbar_init();
-  }
+  if (tid == 0) rows::init_cta(s);
   __syncthreads();
   pdl_enter();  // every thread: inputs and outputs are touched only after this
-  if (p.regsplit) {  // whole warpgroups: warps 0-7 filter; the rest finisher / producer / mirror
+  if (p.regsplit) {  // whole warpgroups: warps 0-7 filter; the rest finisher / producer
     if (warp < rows::kFilterWarps)
       asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(rows::kFilterRegs) : "memory");
-    else if (!clustered)
+    else
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(rows::kOtherRegs) : "memory");
-    else
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(rows::kMirrorRegs) : "memory");
   }
-  if (clustered) {
-    if (warp < rows::kFilterWarps)
-      rows::cluster_filter<T>(s, p, tid);
-    else
-      rows::cluster_mirror<T>(p, tid);
-  } else if (warp < rows::kFilterWarps) {
+  if (warp < rows::kFilterWarps) {
     rows::filter_loop<T>(s, p, tid);
   } else if (warp < rows::kProducerWarp) {
     rows::finish_loop<T>(s, p, tid - rows::kFilterThreads);
   } else if (warp == rows::kProducerWarp && lane == 0) {
     rows::produce_loop<T>(s, p);
   }
+}
+
+// A cluster per row: grid = num_rows * cluster size, 384 threads.
+template <class T>
+__global__ void __launch_bounds__(rows::kThreads) topk_cluster_kernel(const rows::Params p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  rows::Smem& s = *reinterpret_cast<rows::Smem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (tid == 0) rows::init_cta(s);
+  __syncthreads();
+  pdl_enter();  // every thread: inputs and outputs are touched only after this
+  if (p.regsplit) {  // whole warpgroups: warps 0-7 filter; warps 8-11 producer / mirror
+    if (warp < rows::kFilterWarps)
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(rows::kFilterRegs) : "memory");
+    else
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(rows::kMirrorRegs) : "memory");
+  }
+  if (warp < rows::kFilterWarps)
+    rows::cluster_filter<T>(s, p, tid);
+  else
+    rows::cluster_mirror<T>(p, tid);
 }
 
 }  // namespace dsa
