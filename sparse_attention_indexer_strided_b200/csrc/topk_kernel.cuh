@@ -378,6 +378,10 @@ struct FKey {
   const Smem* s;
   __device__ uint32_t operator()(int e) const { return s->fkey[e]; }
 };
+struct FIdx {
+  const Smem* s;
+  __device__ uint32_t operator()(int e) const { return s->fidx[e]; }
+};
 struct FNotIdx {  // larger value = smaller index
   const Smem* s;
   __device__ uint32_t operator()(int e) const { return ~s->fidx[e]; }
@@ -447,8 +451,13 @@ __device__ uint32_t keep_pass(Smem& s, int n, uint32_t A, uint32_t I, int tid, u
 }
 
 // Index cut among the candidates with key == T: the need-th smallest index
-// (1 <= need <= their number).
-__device__ __forceinline__ uint32_t tie_cut(Smem& s, int n, uint32_t T, uint32_t need, int tid) {
+// (1 <= need <= neq, their number; indices are distinct).
+__device__ __forceinline__ uint32_t tie_cut(Smem& s, int n, uint32_t T, uint32_t need, uint32_t neq, int tid) {
+  // when the tied entries' indices form one dense range (a run of one repeated
+  // value, such as a tail of -inf), the need-th smallest is min + need - 1
+  uint32_t lo, hi;
+  filter_minmax(s, n, FIdx{&s}, FKeyIs{&s, T}, lo, hi, tid);
+  if (hi - lo + 1u == neq) return lo + need - 1u;
   return ~filter_kth(s, n, need, FNotIdx{&s}, FKeyIs{&s, T}, tid);
 }
 
@@ -483,7 +492,7 @@ __device__ __noinline__ uint32_t compact_exact(int n, int m, int tid) {
   count_gt_eq(s, n, T, ngt, neq, tid);
   const uint32_t need = static_cast<uint32_t>(m) - ngt;  // entries equal to T that stay
   uint32_t I = 0xFFFFFFFFu;                               // largest index of a kept tie
-  if (neq > need) I = tie_cut(s, n, T, need, tid);
+  if (neq > need) I = tie_cut(s, n, T, need, neq, tid);
   keep_pass<true>(s, n, T, I, tid);
   return T;
 }
@@ -1830,7 +1839,7 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
   const uint32_t ridx = dsmem_map(smem_addr(&s.hidx[0]), 0);
   if (exact && my_keep > 0u) {
     // this rank's share of the tied key: its my_keep lowest indices
-    const uint32_t I = my_keep < q_r ? tie_cut(s, static_cast<int>(n_r), T, my_keep, tid) : 0xFFFFFFFFu;
+    const uint32_t I = my_keep < q_r ? tie_cut(s, static_cast<int>(n_r), T, my_keep, q_r, tid) : 0xFFFFFFFFu;
     keep_pass<true, true>(s, static_cast<int>(n_r), T, I, tid, rkey, ridx, my_off);
   } else {
     keep_pass<false, true>(s, static_cast<int>(n_r), T, 0u, tid, rkey, ridx, my_off);

@@ -132,6 +132,30 @@ def test_cluster_path_many_rows(oracle_mod, dsa):
     assert_parity(oracle_mod, dsa, x, L, 2048)
 
 
+@pytest.mark.parametrize("stride_of_run", [1, 2, 3])
+@pytest.mark.parametrize("shape", ["rows", "cluster"])
+def test_tied_runs_index_cut(oracle_mod, dsa, stride_of_run, shape):
+    """A run of one repeated top value: its copies flood the candidate buffer and
+    the exact compaction cuts them by index. Dense runs (every position) take the
+    dense-range cut (min + need - 1); strided runs take the index select."""
+    rng = np.random.default_rng(3100 + stride_of_run)
+    if shape == "rows":
+        rows, stride, k = 160, 40000, 2048
+    else:
+        rows, stride, k = 3, 600000, 1024
+    x = rng.standard_normal((rows, stride)).astype(np.float32)
+    L = np.full(rows, stride, np.int32)
+    for r in range(rows):
+        a = int(rng.integers(0, stride // 4))
+        b = min(stride, a + stride // 2)
+        x[r, a:b:stride_of_run] = 7.0 if r % 2 else -np.inf
+        if r % 2 == 0:
+            x[r, :] = np.where(np.arange(stride) >= a, x[r], -np.inf)  # -inf tail and run, finite head
+    L[-1] = stride - 5
+    assert (dsa.plan(rows, stride, k)[0] > 1) == (shape == "cluster")
+    assert_parity(oracle_mod, dsa, x, L, k)
+
+
 # --------------------------------------------------------- layout and poison
 @pytest.mark.parametrize("extra,offset", [(0, 0), (1, 0), (2, 1), (3, 3), (5, 2), (256, 0)])
 def test_unaligned_strides_and_bases(oracle_mod, dsa, extra, offset):
