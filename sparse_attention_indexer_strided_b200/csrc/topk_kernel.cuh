@@ -948,9 +948,13 @@ __device__ __forceinline__ void stream_item(Smem& s, Filter& f, RingPos& rp, con
 // m-1 is ranked; the rest of the top m is written in bucket order.
 // NT threads (192: the finisher warps; 256: the filter warps of a cluster's
 // leader) synchronise on named barrier BAR.
-template <int NT, int BAR>
+template <int NT, int BAR, bool kFromFilter = false>
 struct Finisher {
   static constexpr int kWarps = NT / 32;
+  // the candidates: the handover buffer, or (kFromFilter: a CTA's last row)
+  // the filter's own buffer, left in place
+  __device__ __forceinline__ static uint32_t* cand_key(Smem& s) { return kFromFilter ? s.fkey : s.hkey; }
+  __device__ __forceinline__ static uint32_t* cand_idx(Smem& s) { return kFromFilter ? s.fidx : s.hidx; }
   static constexpr int kBuckets = kBucketMax / (4 * NT) * (4 * NT);  // 3840, 4096 or 3584
   static constexpr int kScanPer = kBuckets / NT;  // counters per thread
   static_assert(kBuckets <= kBucketMax && kBuckets >= 2048 && kScanPer % 4 == 0 &&
@@ -983,7 +987,7 @@ struct Finisher {
       const uint32_t q = q0 + lane;
       const bool v = q < qend;
       const uint32_t e = v ? s.perm[q] : 0u;
-      const uint32_t key = v ? s.hkey[e] : 0u, idx = v ? s.hidx[e] : 0xFFFFFFFFu;
+      const uint32_t key = v ? cand_key(s)[e] : 0u, idx = v ? cand_idx(s)[e] : 0xFFFFFFFFu;
       uint32_t s0 = q, s1 = q + 1;  // invalid lanes: a bucket of their own
       if (v) {
         const uint32_t b =
@@ -1006,7 +1010,7 @@ struct Finisher {
         for (uint32_t q2 = s0; q2 < s1; ++q2) {
           if (q2 >= q0 && q2 < q0 + 32u) continue;
           const uint32_t j = s.perm[q2];
-          const uint32_t kj = s.hkey[j], ij = s.hidx[j];
+          const uint32_t kj = cand_key(s)[j], ij = cand_idx(s)[j];
           r += kj > key || (kj == key && ij < idx);
         }
       }
@@ -1058,13 +1062,16 @@ struct Finisher {
   // consecutive places after that digit's running position. (One vote per
   // digit bit, or match.any, costs several times more here.) The masks are
   // zero on entry and on return.
-  // Scratch of the sort passes: the bucket counters, or with more than eight
-  // warps the filter's candidate buffer (free once the candidates sit in hkey).
-  __device__ __forceinline__ static uint32_t* sort_scratch(Smem& s) { return kWarps > kFilterWarps ? s.fkey : s.bcnt; }
+  // Scratch of the sort passes: the bucket counters; with more than eight
+  // warps, the handover buffer (hkey and hidx, contiguous) when the candidates
+  // stay in the filter's buffer, else the filter's buffer.
+  __device__ __forceinline__ static uint32_t* sort_scratch(Smem& s) {
+    return kWarps > kFilterWarps ? (kFromFilter ? s.hkey : s.fkey) : s.bcnt;
+  }
   __device__ __forceinline__ static void radix_passes(Smem& s, int n, uint32_t kmax, int half, uint32_t vary,
                                                       uint16_t*& pa, uint16_t*& pb, int fid) {
     constexpr int kBins = 256;
-    static_assert(kWarps * kBins + kWarps * kBins / 2 + kBins <= (kWarps > kFilterWarps ? kFiltCap : kBucketMax) &&
+    static_assert(kWarps * kBins + kWarps * kBins / 2 + kBins <= (kWarps > kFilterWarps ? 2 * kHandCap : kBucketMax) &&
                       kHandCap < 65536,
                   "lane masks, 16-bit digit counters and digit starts fit the sort scratch");
     const int fw = fid >> 5, lane = fid & 31;
@@ -1097,7 +1104,7 @@ struct Finisher {
       const int p0 = pos[0];
       const bool run = ((dm >> p0) & ((dm >> p0) + 1u)) == 0u;  // the bits are contiguous
       auto digit = [&](uint32_t e) -> uint32_t {
-        const uint32_t x = half ? kmax - s.hkey[e] : s.hidx[e];
+        const uint32_t x = half ? kmax - cand_key(s)[e] : cand_idx(s)[e];
         if (run) return (x >> p0) & (dm >> p0);
         uint32_t d = 0u;
 #pragma unroll
@@ -1216,8 +1223,8 @@ struct Finisher {
       bool keep = false;
       uint32_t hi = 0u, lo = 0u;
       if (e < n) {
-        hi = kmax - s.hkey[e];
-        lo = s.hidx[e];
+        hi = kmax - cand_key(s)[e];
+        lo = cand_idx(s)[e];
         keep = ((static_cast<uint64_t>(hi) << 32) | lo) <= cut;
       }
       const uint32_t b = __ballot_sync(kFull, keep);
@@ -1264,16 +1271,16 @@ struct Finisher {
     }
     const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
     if (fid == 0) {
-      if (m == k) s.rec[0] = s.hkey[pa[k - 1]];
-      if (a < m) s.rec[1] = s.hkey[pa[a]];
+      if (m == k) s.rec[0] = cand_key(s)[pa[k - 1]];
+      if (a < m) s.rec[1] = cand_key(s)[pa[a]];
     }
     // the sorted order's first m indices (the permutation buffer may be the
     // output stage, so it is read, not staged)
     if (p.table == nullptr) {
-      for (int q = fid; q < m; q += NT) o[q] = static_cast<int32_t>(s.hidx[pa[q]]);
+      for (int q = fid; q < m; q += NT) o[q] = static_cast<int32_t>(cand_idx(s)[pa[q]]);
     } else {
       const int32_t* trow = p.table + row * p.table_stride;
-      for (int q = fid; q < m; q += NT) o[q] = __ldg(trow + s.hidx[pa[q]]);
+      for (int q = fid; q < m; q += NT) o[q] = __ldg(trow + cand_idx(s)[pa[q]]);
     }
     bar();
   }
@@ -1289,13 +1296,13 @@ struct Finisher {
     for (int q = m + fid; q < k; q += NT) o[q] = -1;
     if (n <= 0) return;
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, imax = 0u, kdiff = 0u;
-    const uint32_t key0 = s.hkey[0];
+    const uint32_t key0 = cand_key(s)[0];
     for (int e = fid; e < n; e += NT) {
-      const uint32_t key = s.hkey[e];
+      const uint32_t key = cand_key(s)[e];
       kmin = min(kmin, key);
       kmax = max(kmax, key);
       kdiff |= key ^ key0;
-      imax = max(imax, s.hidx[e]);
+      imax = max(imax, cand_idx(s)[e]);
     }
     kmin = __reduce_min_sync(kFull, kmin);
     kmax = __reduce_max_sync(kFull, kmax);
@@ -1332,7 +1339,7 @@ struct Finisher {
       for (int i = 0; i < kScanPer / 4; ++i) bc4[i] = make_uint4(0u, 0u, 0u, 0u);
       bar();
       for (int e = fid; e < n; e += NT) {
-        const uint64_t c = comp(s.hkey[e], s.hidx[e]);
+        const uint64_t c = comp(cand_key(s)[e], cand_idx(s)[e]);
         if (c <= cmax) atomicAdd(&s.bcnt[static_cast<uint32_t>(c >> sh)], 1u);
       }
       bar();
@@ -1409,7 +1416,7 @@ struct Finisher {
       return;
     }
     for (int e = fid; e < n; e += NT) {
-      const uint64_t cc = comp(s.hkey[e], s.hidx[e]);
+      const uint64_t cc = comp(cand_key(s)[e], cand_idx(s)[e]);
       if (cc > cmax) continue;
       const uint32_t q = atomicAdd(&s.bcnt[static_cast<uint32_t>(cc >> sh)], 1u);
       s.perm[q] = static_cast<uint16_t>(e);
@@ -1429,16 +1436,16 @@ struct Finisher {
       const uint32_t s0 = bm ? s.bcnt[bm - 1] : 0u, s1 = s.bcnt[bm];
       for (uint32_t q = fid; q < s0; q += NT) {
         const uint32_t e = s.perm[q];
-        s.ostage[q] = static_cast<int32_t>(s.hidx[e]);
-        if (q == static_cast<uint32_t>(a)) s.rec[1] = s.hkey[e];
+        s.ostage[q] = static_cast<int32_t>(cand_idx(s)[e]);
+        if (q == static_cast<uint32_t>(a)) s.rec[1] = cand_key(s)[e];
       }
       for (uint32_t q = s0 + fid; q < s1; q += NT) {
         const uint32_t e = s.perm[q];
-        const uint32_t key = s.hkey[e], idx = s.hidx[e];
+        const uint32_t key = cand_key(s)[e], idx = cand_idx(s)[e];
         uint32_t r = s0;
         for (uint32_t q2 = s0; q2 < s1; ++q2) {
           const uint32_t j = s.perm[q2];
-          const uint32_t kj = s.hkey[j], ij = s.hidx[j];
+          const uint32_t kj = cand_key(s)[j], ij = cand_idx(s)[j];
           r += kj > key || (kj == key && ij < idx);
         }
         if (r < static_cast<uint32_t>(m)) {
@@ -1450,7 +1457,7 @@ struct Finisher {
     } else {
       // each candidate: its bucket's start plus the bucket members ahead of it
       for (int e = fid; e < n; e += NT) {
-        const uint32_t key = s.hkey[e], idx = s.hidx[e];
+        const uint32_t key = cand_key(s)[e], idx = cand_idx(s)[e];
         const uint64_t cc = comp(key, idx);
         if (cc > cmax) continue;
         const uint32_t b = static_cast<uint32_t>(cc >> sh);
@@ -1459,7 +1466,7 @@ struct Finisher {
         uint32_t r = s0;
         for (uint32_t q = s0; q < s1; ++q) {
           const uint32_t j = s.perm[q];
-          const uint32_t kj = s.hkey[j], ij = s.hidx[j];
+          const uint32_t kj = cand_key(s)[j], ij = cand_idx(s)[j];
           r += kj > key || (kj == key && ij < idx);
         }
         if (r < static_cast<uint32_t>(m)) {
@@ -1478,7 +1485,7 @@ using RowFinisher = Finisher<kFinishThreads, 2>;
 // the filter warps' own ranking of a cluster leader's row
 using LeaderFinisher = Finisher<kFilterThreads, 1>;
 // a CTA's last row, ranked by the filter and finisher warps together
-using JointFinisher = Finisher<kJointThreads, 3>;
+using JointFinisher = Finisher<kJointThreads, 3, true>;
 
 // Where the filter and finisher warps meet after their row loops. Both roles reach it on every path (a wait that gave up ends a
 // loop early; no loop ends without passing here), so the hardware barrier
@@ -1560,19 +1567,12 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
         s.own_len = L;
       }
     }
-    bar_filter();  // the own estimate is read at the next row's start
-    // hand over: wait until the finishers released the previous handover (a
-    // wait that gave up hands over regardless; the row's output is undefined)
-    mbar_wait_sleep(&s.hempty, (h & 1) ^ 1, &s.wait);
-    for (int e = tid; e < static_cast<int>(f.cnt); e += kFilterThreads) {
-      s.hkey[e] = s.fkey[e];
-      s.hidx[e] = s.fidx[e];
-    }
+    bar_filter();  // the own estimate is read at the next row's start; every append is visible
     if (row + gridDim.x >= p.num_rows) {
-      // the CTA's last row: the finisher warps have stopped after the row
-      // before it, and nothing else is left to stream. The only row: both
-      // roles rank it after the rendezvous. Else the filter warps rank it
-      // (no handover latency, in parallel with the finisher warps' last row).
+      // the CTA's last row: the finisher warps stop after the row before it
+      // and nothing else is left to stream, so both roles rank this one
+      // together after the rendezvous, from the filter's buffer (more
+      // threads, no handover copy)
       if (tid == 0) {
         s.h_row = row;
         s.h_n = static_cast<int32_t>(f.cnt);
@@ -1580,6 +1580,13 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
         s.joint = 1u;
       }
       break;
+    }
+    // hand over: wait until the finishers released the previous handover (a
+    // wait that gave up hands over regardless; the row's output is undefined)
+    mbar_wait_sleep(&s.hempty, (h & 1) ^ 1, &s.wait);
+    for (int e = tid; e < static_cast<int>(f.cnt); e += kFilterThreads) {
+      s.hkey[e] = s.fkey[e];
+      s.hidx[e] = s.fidx[e];
     }
     if (tid == 0) {
       s.h_row = row;
