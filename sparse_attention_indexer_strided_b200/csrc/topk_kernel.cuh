@@ -978,8 +978,9 @@ struct Finisher {
   // neighbouring lanes by shuffles (only as far as the widest bucket of the
   // window), the few beyond the window from shared memory. In set mode only
   // the bucket holding rank m-1 is ranked; earlier positions stay as they lie.
+  template <class Bucket>
   __device__ __forceinline__ static void rank_by_windows(Smem& s, int n, int m, int k, int a, uint32_t bm,
-                                                         bool set_mode, uint32_t kmax, int sh, int fid) {
+                                                         bool set_mode, Bucket bucket_of, int fid) {
     const int fw = fid >> 5, lane = fid & 31;
     const uint32_t qend = s.bcnt[bm];  // positions past this have rank >= m
     const uint32_t cut0 = bm ? s.bcnt[bm - 1] : 0u;
@@ -990,8 +991,8 @@ struct Finisher {
       const uint32_t key = v ? cand_key(s)[e] : 0u, idx = v ? cand_idx(s)[e] : 0xFFFFFFFFu;
       uint32_t s0 = q, s1 = q + 1;  // invalid lanes: a bucket of their own
       if (v) {
-        const uint32_t b =
-            static_cast<uint32_t>((((static_cast<uint64_t>(kmax - key)) << 32) | idx) >> sh);
+        uint32_t b;
+        bucket_of(key, idx, b);
         s0 = b ? s.bcnt[b - 1] : 0u;
         s1 = s.bcnt[b];
       }
@@ -1331,6 +1332,32 @@ struct Finisher {
     auto comp = [&](uint32_t key, uint32_t idx) -> uint64_t {
       return (static_cast<uint64_t>(kmax - key) << 32) | idx;
     };
+    // A row ranked alone (its latency is the kernel's tail) takes a first
+    // pass that buckets linearly in the value when the keys are off a coarse
+    // grid and their range is finite: smooth logits then rarely need a second
+    // pass, where 12-bit slices of a key range spanning both signs
+    // crowd most values into a few buckets. Still exact: the bucket is a
+    // monotone function of the key (correctly rounded steps), and the members
+    // of one bucket are ranked by comparison. A first pass that leaves a
+    // bucket crowded hands over to the slices of the composite.
+    const float vtop = from_key(kmax), vlow = from_key(kmin);
+    float scale = 0.f;
+    bool lin = alone && grid < 8 && vtop > vlow && isfinite(vtop) && isfinite(vlow);
+    if (lin) {
+      scale = static_cast<float>(kBuckets - 1) / (vtop - vlow);
+      lin = isfinite(scale) && scale > 0.f;
+    }
+    // bucket b of a candidate; false: past the range counted (after bm)
+    auto bucket_of = [&](uint32_t key, uint32_t idx, uint32_t& b) -> bool {
+      if (lin) {
+        const float d = (vtop - from_key(key)) * scale;
+        b = d < static_cast<float>(kBuckets - 1) ? static_cast<uint32_t>(d) : static_cast<uint32_t>(kBuckets - 1);
+        return true;
+      }
+      const uint64_t c = comp(key, idx);
+      b = static_cast<uint32_t>(c >> sh);
+      return c <= cmax;
+    };
     uint4* bc4 = reinterpret_cast<uint4*>(&s.bcnt[fid * kScanPer]);
     const uint32_t mm1 = static_cast<uint32_t>(m - 1);
     uint32_t big = 0;
@@ -1339,8 +1366,8 @@ struct Finisher {
       for (int i = 0; i < kScanPer / 4; ++i) bc4[i] = make_uint4(0u, 0u, 0u, 0u);
       bar();
       for (int e = fid; e < n; e += NT) {
-        const uint64_t c = comp(cand_key(s)[e], cand_idx(s)[e]);
-        if (c <= cmax) atomicAdd(&s.bcnt[static_cast<uint32_t>(c >> sh)], 1u);
+        uint32_t b;
+        if (bucket_of(cand_key(s)[e], cand_idx(s)[e], b)) atomicAdd(&s.bcnt[b], 1u);
       }
       bar();
       // exclusive scan: thread fid owns counters [kScanPer fid, kScanPer (fid + 1))
@@ -1400,8 +1427,14 @@ struct Finisher {
       // pass holds values on a coarse grid (equal keys), which finer slices of
       // the same composite range do not split: sort instead (the first pass
       // alone can be coarse when the keys span both signs)
-      if (big <= static_cast<uint32_t>(kSmallBucket) ||
-          (big > static_cast<uint32_t>(kBigBucket) && (pass >= 1 || sh <= 32 + grid)) || sh == 0 ||
+      if (big <= static_cast<uint32_t>(kSmallBucket)) break;
+      if (lin) {  // crowded after the value-linear pass: the composite slices from the start
+        lin = false;
+        pass = -1;
+        bar();  // bc[4] and nred[4] are rewritten by the next pass
+        continue;
+      }
+      if ((big > static_cast<uint32_t>(kBigBucket) && (pass >= 1 || sh <= 32 + grid)) || sh == 0 ||
           pass == kSortPasses - 1)
         break;
       cmax = ((static_cast<uint64_t>(bm) + 1u) << sh) - 1u;
@@ -1416,9 +1449,9 @@ struct Finisher {
       return;
     }
     for (int e = fid; e < n; e += NT) {
-      const uint64_t cc = comp(cand_key(s)[e], cand_idx(s)[e]);
-      if (cc > cmax) continue;
-      const uint32_t q = atomicAdd(&s.bcnt[static_cast<uint32_t>(cc >> sh)], 1u);
+      uint32_t b;
+      if (!bucket_of(cand_key(s)[e], cand_idx(s)[e], b)) continue;
+      const uint32_t q = atomicAdd(&s.bcnt[b], 1u);
       s.perm[q] = static_cast<uint16_t>(e);
     }
     bar();  // bcnt[b] is now the end of bucket b (= start of b + 1)
@@ -1429,7 +1462,7 @@ struct Finisher {
       // nothing overlaps this row, and most candidates rank past m: ranking
       // only the positions before m is fastest (the per-candidate loop below
       // takes the fewest issue slots, which counts while rows still stream)
-      rank_by_windows(s, n, m, k, a, bm, set_mode, kmax, sh, fid);
+      rank_by_windows(s, n, m, k, a, bm, set_mode, bucket_of, fid);
     } else if (set_mode) {
       // set mode: positions before the bucket holding rank m-1 are taken as
       // they lie (bucket order); only that bucket's members are ranked
@@ -1458,9 +1491,8 @@ struct Finisher {
       // each candidate: its bucket's start plus the bucket members ahead of it
       for (int e = fid; e < n; e += NT) {
         const uint32_t key = cand_key(s)[e], idx = cand_idx(s)[e];
-        const uint64_t cc = comp(key, idx);
-        if (cc > cmax) continue;
-        const uint32_t b = static_cast<uint32_t>(cc >> sh);
+        uint32_t b;
+        if (!bucket_of(key, idx, b)) continue;
         const uint32_t s0 = b ? s.bcnt[b - 1] : 0u, s1 = s.bcnt[b];
         if (s0 >= static_cast<uint32_t>(m)) continue;
         uint32_t r = s0;
