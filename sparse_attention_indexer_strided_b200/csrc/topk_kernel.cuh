@@ -1635,15 +1635,16 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
 
 
 // The estimate the filter starts a later row from: the k-th value minus half
-// the gap to the 3k/4-th, and at least one step of the element type's value
-// grid below the k-th (a coarse grid, such as bf16 logits, often puts both
-// ranks on one value; an estimate equal to the k-th value then lets too few
-// values of a similar row through and forces a re-read).
+// the gap to the 3k/4-th, and at least one step (two for 16-bit values) of
+// the element type's value grid below the k-th (a coarse grid, such as bf16
+// logits, often puts both ranks on one value; an estimate equal to the k-th
+// value then lets too few values of a similar row through and forces a
+// re-read).
 template <class T>
 __device__ __forceinline__ float row_estimate(float vt, float va) {
   constexpr int kMantissa = sizeof(T) == 4 ? 23 : (Elem<T>::kCode == DSA_DTYPE_BF16 ? 7 : 10);
   const float step = fabsf(vt) * (1.0f / static_cast<float>(1 << kMantissa));
-  return vt - fmaxf(0.5f * (va - vt), step);
+  return vt - fmaxf(0.5f * (va - vt), (sizeof(T) == 4 ? 1.0f : 2.0f) * step);
 }
 
 template <class T>
