@@ -744,24 +744,25 @@ __device__ __forceinline__ Filter refilter_from_global(Smem& s, Filter f, RowSpa
 
 // The need-th largest of the kSampleVals sampled keys in fkey, to within
 // one bin of a second histogram round (1 <= need <= the number sampled; every
-// sampled key lies in [lo, hi]). Round one counts 4096 bins over a 12-bit
+// sampled key lies in [lo, hi]). Round one counts 1024 bins over a 10-bit
 // slice of [lo, hi] below its highest differing bit and finds, from the top,
 // the bin holding the need-th key; round two does the same inside that bin.
 // The result is the smallest sampled key in the final bin: at least `need`
 // sampled keys are at or above it, and at most the rest of that bin besides
-// (for fp32 logits the second round's bins are a few units in the last place
-// wide; for values on a coarse grid the bin is one value, the exact answer).
+// (for fp32 logits a second-round bin spans about 1e-3 of the value and holds
+// about one sampled key; for values on a coarse grid it is one value, the
+// exact answer).
 // Counters live in fidx, unused until the item streams. Two plain-atomic
 // passes instead of a radix select's three or four rounds with their
 // barriers.
 __device__ __forceinline__ uint32_t sample_kth(Smem& s, uint32_t need, uint32_t lo, uint32_t hi, int tid) {
-  constexpr int kBins = 4096, kPer = kBins / kFilterThreads;  // 16 bins per thread
+  constexpr int kBits = 10, kBins = 1 << kBits, kPer = kBins / kFilterThreads;  // 4 bins per thread
   const int w = tid >> 5, lane = tid & 31;
   uint32_t* hist = s.fidx;
   const uint32_t span = hi - lo;
   if (span == 0u) return lo;
   const int bits = 32 - __clz(span);
-  int sh = bits > 12 ? bits - 12 : 0;  // (key - lo) >> sh < 4096
+  int sh = bits > kBits ? bits - kBits : 0;  // (key - lo) >> sh < kBins
   uint32_t base = lo, top = hi;
   for (int round = 0; round < 2; ++round) {
     uint4* h4 = reinterpret_cast<uint4*>(hist + kPer * tid);
@@ -811,7 +812,7 @@ __device__ __forceinline__ uint32_t sample_kth(Smem& s, uint32_t need, uint32_t 
     base += b << sh;
     top = min(top, base + ((1u << sh) - 1u));
     if (round == 1 || sh == 0) break;
-    sh = sh > 12 ? sh - 12 : 0;
+    sh = sh > kBits ? sh - kBits : 0;
     bar_filter();  // bc and the counters are rewritten by the next round
   }
   // the smallest sampled key in the final bin: a key that occurs (a value
