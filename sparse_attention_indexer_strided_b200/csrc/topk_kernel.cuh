@@ -163,6 +163,8 @@ struct __align__(128) Smem {
   uint32_t abort_any;  // cluster mode: some rank gave up (read by the leader)
   uint32_t final_bar;  // cluster mode: number of cluster barriers of the merge (0: not yet known)
   uint32_t joint;      // many-row mode: the CTA's last row is ranked by filter and finisher warps together
+  uint32_t merge_bars; // cluster mode: cluster barriers of earlier merge attempts
+  uint32_t merge_retry;
   unsigned long long full[kMaxStages], empty[kMaxStages];
   unsigned long long hfull, hempty;
 };
@@ -1736,11 +1738,13 @@ __device__ void produce_loop(Smem& s, const Params& p) {
 // of every rank run the merge; at the leader (rank 0) the survivors end in
 // hkey/hidx. Returns the number gathered there. The producer warp mirrors
 // every cluster barrier (s.final_bar tells it how many there are).
-__device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool aborted, uint32_t rank,
+constexpr uint32_t kMergeRetry = 0xFFFFFFFFu;
+
+__device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool aborted, bool open, uint32_t rank,
                                                uint32_t ncta, int tid) {
   Smem& s = cta_smem();
   const int w = tid >> 5, lane = tid & 31;
-  uint32_t nbar = 0;
+  uint32_t nbar = s.merge_bars;
   uint32_t* phist = s.bcnt;        // [2][256], per rank, read by the others
   uint32_t* ghist = s.bcnt + 512;  // [256], cluster sums
   // ---- phase 1: publish (count, min key, max key, gave up) of this rank
@@ -1751,17 +1755,19 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
     s.pub[1] = mn;
     s.pub[2] = mx;
     s.pub[3] = aborted ? 1u : 0u;
+    s.pub[6] = open ? 1u : 0u;
   }
   cluster_barrier();
   ++nbar;
   if (w == 0) {
-    uint32_t n = 0, lo_r = 0xFFFFFFFFu, hi_r = 0u, ab = 0u;
+    uint32_t n = 0, lo_r = 0xFFFFFFFFu, hi_r = 0u, ab = 0u, op = 0u;
     if (lane < static_cast<int>(ncta)) {
       const uint32_t a = dsmem_map(smem_addr(&s.pub[0]), lane);
       n = dsmem_ld(a);
       lo_r = dsmem_ld(a + 4);
       hi_r = dsmem_ld(a + 8);
       ab = dsmem_ld(a + 12);
+      op = dsmem_ld(a + 24);
     }
     const bool full_rank = lane < static_cast<int>(ncta) && n >= m;
     const uint32_t N = __reduce_add_sync(kFull, n);
@@ -1771,19 +1777,31 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
     const uint32_t B = __reduce_max_sync(kFull, full_rank ? lo_r : 0u);
     const bool any_full = __ballot_sync(kFull, full_rank) != 0;
     const bool any_ab = __ballot_sync(kFull, ab != 0u) != 0;
+    const bool any_open = __ballot_sync(kFull, op != 0u) != 0;
     if (lane == 0) {
       s.bc[2] = N;
       s.bc[3] = any_full ? B : gmin;
       s.bc[4] = gmax;
       s.bc[5] = gmin;
       s.abort_any = any_ab ? 1u : 0u;
+      // fewer than m candidates, and some rank left out its -inf values: they
+      // are needed, so every rank takes its chunk again with no threshold
+      s.merge_retry = (any_open && N < m && !any_ab) ? 1u : 0u;
     }
   }
   bar_filter();
   const uint32_t N = s.bc[2];
   uint32_t lo = s.bc[3], hi = s.bc[4];
   const uint32_t gmin = s.bc[5];
+  const bool retry = s.merge_retry != 0u;
   bar_filter();
+  if (retry) {
+    cluster_barrier();  // every rank has read the published values before they change
+    ++nbar;
+    if (tid == 0) s.merge_bars = nbar;
+    bar_filter();
+    return kMergeRetry;
+  }
   uint32_t need = m;
   bool exact = false;
   if (N <= static_cast<uint32_t>(kHandCap)) {
@@ -1830,7 +1848,7 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
       if (S <= static_cast<uint32_t>(kHandCap)) break;
     }
   }
-  if (tid == 0) s.final_bar = nbar + 2;  // phases 3 and 4 end with one cluster barrier each
+  if (tid == 0) s.final_bar = nbar + 2;  // phases 3 and 4 end with one cluster barrier each (counted from the first attempt)
   // ---- phase 3: publish this rank's survivor counts
   // exact: keep key > T plus a rank-ordered share of key == T; else keep key >= lo
   const uint32_t T = exact ? lo : lo - 1u;
@@ -1964,6 +1982,13 @@ __device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid
       f.t = ts;
     }
   }
+  // With no sampled threshold the rank keeps only values above -inf: a chunk
+  // of -inf (a row's padded tail) would otherwise fill the buffer with ties
+  // and cut them by index while the other ranks wait at the merge. The merge
+  // takes the chunks again with no threshold if the row turns out to hold
+  // fewer than m values above -inf.
+  const bool open = !spec;
+  if (open) f.t = __int_as_float(0xff7fffff);  // -FLT_MAX: keep x unless x < -FLT_MAX, i.e. x = -inf
   f.cnt = 0;
   f.compacted = false;
   f.strict = false;
@@ -1980,7 +2005,12 @@ __device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid
     }
     if (f.cnt > static_cast<uint32_t>(kHandCap)) compact_any(s, f, static_cast<int>(m_r), tid);
   }
-  const uint32_t total = cluster_merge(f.cnt, it.m, !ok, it.rank, it.ncta, tid);
+  uint32_t total = cluster_merge(f.cnt, it.m, !ok, open, it.rank, it.ncta, tid);
+  if (total == kMergeRetry) {  // the same on every rank of the cluster
+    f = refilter_from_global<T>(s, f, sp, Lc, static_cast<uint32_t>(it.c0), static_cast<int>(m_r), tid);
+    if (f.cnt > static_cast<uint32_t>(kHandCap)) compact_any(s, f, static_cast<int>(m_r), tid);
+    total = cluster_merge(f.cnt, it.m, !ok, false, it.rank, it.ncta, tid);
+  }
   if (it.rank != 0) return;
   if (s.abort_any) {  // some rank gave up: no valid result for this row
     for (int q = tid; q < k; q += kFilterThreads) p.out[it.row * static_cast<int64_t>(k) + q] = -1;
@@ -2010,6 +2040,8 @@ __device__ __forceinline__ void init_cta(Smem& s) {
   s.abort_any = 0u;
   s.final_bar = 0u;
   s.joint = 0u;
+  s.merge_bars = 0u;
+  s.merge_retry = 0u;
   fence_mbar_init();
 }
 

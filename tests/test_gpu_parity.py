@@ -156,6 +156,28 @@ def test_tied_runs_index_cut(oracle_mod, dsa, stride_of_run, shape):
     assert_parity(oracle_mod, dsa, x, L, k)
 
 
+@pytest.mark.parametrize("k", [1024, 2048])
+def test_cluster_rows_mostly_neg_inf(oracle_mod, dsa, k):
+    """Cluster ranks with no sampled threshold leave out -inf values; rows with
+    fewer than k values above -inf send every rank back over its chunk with no
+    threshold. Rows: a few finite values, all -inf, -inf in every other half of
+    the chunks, and a normal row with a -inf tail."""
+    rng = np.random.default_rng(3300 + k)
+    stride = 600000
+    L = np.array([stride, stride, stride, stride - 7, 250000], np.int32)
+    x = np.full((len(L), stride), -np.inf, np.float32)
+    pos = rng.choice(stride, size=500, replace=False)
+    x[0, pos] = rng.standard_normal(500).astype(np.float32)
+    # row 1: all -inf
+    chunk = stride // 16
+    for c in range(0, 16, 2):
+        x[2, c * chunk:(c + 1) * chunk] = rng.standard_normal(chunk).astype(np.float32)
+    x[3, : stride // 2] = rng.standard_normal(stride // 2).astype(np.float32)
+    x[4, : 1500] = np.round(rng.standard_normal(1500) * 2).astype(np.float32) / 2
+    assert dsa.plan(len(L), stride, k)[0] > 1
+    assert_parity(oracle_mod, dsa, x, L, k)
+
+
 # --------------------------------------------------------- layout and poison
 @pytest.mark.parametrize("extra,offset", [(0, 0), (1, 0), (2, 1), (3, 3), (5, 2), (256, 0)])
 def test_unaligned_strides_and_bases(oracle_mod, dsa, extra, offset):
