@@ -1739,6 +1739,7 @@ __device__ void produce_loop(Smem& s, const Params& p) {
 // hkey/hidx. Returns the number gathered there. The producer warp mirrors
 // every cluster barrier (s.final_bar tells it how many there are).
 constexpr uint32_t kMergeRetry = 0xFFFFFFFFu;
+constexpr int kMaxClusterSize = 16;  // the largest cluster the host plans
 
 __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool aborted, bool open, uint32_t rank,
                                                uint32_t ncta, int tid) {
@@ -1824,9 +1825,16 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
       cluster_barrier();
       ++nbar;
       {
+        // every rank's count for this thread's bin: the remote loads are all
+        // issued before any is summed (one at a time, each load's round trip
+        // would add up across the cluster)
         const uint32_t a = smem_addr(&ph[tid]);
+        uint32_t v[kMaxClusterSize];
+#pragma unroll
+        for (int r = 0; r < kMaxClusterSize; ++r) v[r] = static_cast<uint32_t>(r) < ncta ? dsmem_ld(dsmem_map(a, r)) : 0u;
         uint32_t g = 0;
-        for (uint32_t r = 0; r < ncta; ++r) g += dsmem_ld(dsmem_map(a, r));
+#pragma unroll
+        for (int r = 0; r < kMaxClusterSize; ++r) g += v[r];
         ghist[tid] = g;
       }
       bar_filter();
