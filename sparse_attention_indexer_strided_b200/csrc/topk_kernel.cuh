@@ -397,14 +397,53 @@ struct FKeyIs {
   __device__ bool operator()(int e) const { return s->fkey[e] == T; }
 };
 
+// Stores the candidates with key > A and, when kTies, those with key == A and
+// index <= I at positions off.. of the shared::cluster addresses rkey / ridx
+// (the copy to a cluster's leader, another buffer). Two rolled passes over the
+// candidates, count then store, instead of holding 32 entries per thread in
+// registers: it runs once per launch, so its code size is its cost. Returns
+// the kept count (uniform).
+template <bool kTies>
+__device__ uint32_t keep_remote(Smem& s, int n, uint32_t A, uint32_t I, int tid, uint32_t rkey, uint32_t ridx,
+                                uint32_t off) {
+  const int w = tid >> 5, lane = tid & 31;
+  auto kept = [&](int e) -> bool {
+    const uint32_t kk = s.fkey[e];
+    return kk > A || (kTies && kk == A && s.fidx[e] <= I);
+  };
+  uint32_t nk = 0;
+  for (int e = tid; e < n; e += kFilterThreads) nk += kept(e) ? 1u : 0u;
+  uint32_t incl = nk;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) s.fred[0][w] = incl;
+  bar_filter();
+  uint32_t pos = incl - nk, total = 0;
+#pragma unroll
+  for (int ww = 0; ww < kFilterWarps; ++ww) {
+    const uint32_t c = s.fred[0][ww];
+    pos += ww < w ? c : 0u;
+    total += c;
+  }
+  for (int e = tid; e < n; e += kFilterThreads) {
+    if (kept(e)) {
+      dsmem_st(rkey + 4u * (off + pos), s.fkey[e]);
+      dsmem_st(ridx + 4u * (off + pos), s.fidx[e]);
+      ++pos;
+    }
+  }
+  bar_filter();
+  return total;
+}
+
 // Keeps the candidates with key > A and, when kTies, those with key == A and
-// index <= I: in place and in any order (local), or stored at positions
-// off.. of the shared::cluster addresses rkey / ridx (remote, cluster mode).
-// Every filter thread reads its entries before any is written. Returns the
-// kept count (uniform).
-template <bool kTies, bool kRemote = false>
-__device__ uint32_t keep_pass(Smem& s, int n, uint32_t A, uint32_t I, int tid, uint32_t rkey = 0u, uint32_t ridx = 0u,
-                              uint32_t off = 0u) {
+// index <= I, in place and in any order. Every filter thread reads its entries
+// (into registers) before any is written. Returns the kept count (uniform).
+template <bool kTies>
+__device__ uint32_t keep_pass(Smem& s, int n, uint32_t A, uint32_t I, int tid) {
   const int w = tid >> 5, lane = tid & 31;
   uint32_t kk[kPerThread], ii[kPerThread], keep = 0;
 #pragma unroll
@@ -438,13 +477,8 @@ __device__ uint32_t keep_pass(Smem& s, int n, uint32_t A, uint32_t I, int tid, u
 #pragma unroll
   for (int it = 0; it < kPerThread; ++it) {
     if ((keep >> it) & 1u) {
-      if (kRemote) {
-        dsmem_st(rkey + 4u * (off + pos), kk[it]);
-        dsmem_st(ridx + 4u * (off + pos), ii[it]);
-      } else {
-        s.fkey[pos] = kk[it];
-        s.fidx[pos] = ii[it];
-      }
+      s.fkey[pos] = kk[it];
+      s.fidx[pos] = ii[it];
       ++pos;
     }
   }
@@ -1907,9 +1941,9 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
   if (exact && my_keep > 0u) {
     // this rank's share of the tied key: its my_keep lowest indices
     const uint32_t I = my_keep < q_r ? tie_cut(s, static_cast<int>(n_r), T, my_keep, q_r, tid) : 0xFFFFFFFFu;
-    keep_pass<true, true>(s, static_cast<int>(n_r), T, I, tid, rkey, ridx, my_off);
+    keep_remote<true>(s, static_cast<int>(n_r), T, I, tid, rkey, ridx, my_off);
   } else {
-    keep_pass<false, true>(s, static_cast<int>(n_r), T, 0u, tid, rkey, ridx, my_off);
+    keep_remote<false>(s, static_cast<int>(n_r), T, 0u, tid, rkey, ridx, my_off);
   }
   cluster_barrier();
   ++nbar;
