@@ -1089,9 +1089,9 @@ struct Finisher {
     }
   }
 
-  // One stable LSD pass per digit of up to eight of the bits `vary` of one
-  // half of C (half 0: the index, half 1: kmax - key), lowest bits first,
-  // moving the permutation from *pa to *pb and swapping them. Each warp owns a contiguous range of the
+  // One stable LSD pass per digit of up to eight of the bits `vary` of the
+  // composite C = (kmax - key) << 32 | index, lowest bits first, moving the
+  // permutation from *pa to *pb and swapping them. Each warp owns a contiguous range of the
   // current order. Counting needs no order: every lane adds one to its
   // warp's counter for its digit (16-bit counters, two to a word). The
   // scatter walks the warp's chunks of 32 in order; the lanes holding one
@@ -1106,7 +1106,7 @@ struct Finisher {
   __device__ __forceinline__ static uint32_t* sort_scratch(Smem& s) {
     return kWarps > kFilterWarps ? (kFromFilter ? s.hkey : s.fkey) : s.bcnt;
   }
-  __device__ __forceinline__ static void radix_passes(Smem& s, int n, uint32_t kmax, int half, uint32_t vary,
+  __device__ __forceinline__ static void radix_passes(Smem& s, int n, uint32_t kmax, uint64_t vary,
                                                       uint16_t*& pa, uint16_t*& pb, int fid) {
     constexpr int kBins = 256;
     static_assert(kWarps * kBins + kWarps * kBins / 2 + kBins <= (kWarps > kFilterWarps ? 2 * kHandCap : kBucketMax) &&
@@ -1123,18 +1123,19 @@ struct Finisher {
     const int per = ((n + kWarps - 1) / kWarps + 31) & ~31;  // items per warp, whole chunks
     const int i0 = fw * per, i1 = min(n, i0 + per);
     const uint32_t lt = lanemask_lt();
-    uint32_t rest = vary;
+    uint64_t rest = vary;
     while (rest != 0u) {
-      // this pass's digit: the next eight (or fewer) bits that vary, lowest
-      // first; bits that are the same in every candidate do not order them
-      uint32_t dm = 0u;
+      // this pass's digit: the next eight (or fewer) bits of C that vary,
+      // lowest first, across both halves (bits that are the same in every
+      // candidate do not order them)
+      uint64_t dm = 0u;
       int pos[8], nb = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         pos[i] = 0;
         if (rest != 0u) {
-          pos[i] = __ffs(rest) - 1;
-          dm |= 1u << pos[i];
+          pos[i] = __ffsll(static_cast<long long>(rest)) - 1;
+          dm |= 1ull << pos[i];
           rest &= rest - 1u;
           ++nb;
         }
@@ -1142,12 +1143,12 @@ struct Finisher {
       const int p0 = pos[0];
       const bool run = ((dm >> p0) & ((dm >> p0) + 1u)) == 0u;  // the bits are contiguous
       auto digit = [&](uint32_t e) -> uint32_t {
-        const uint32_t x = half ? kmax - cand_key(s)[e] : cand_idx(s)[e];
-        if (run) return (x >> p0) & (dm >> p0);
+        const uint64_t x = (static_cast<uint64_t>(kmax - cand_key(s)[e]) << 32) | cand_idx(s)[e];
+        if (run) return static_cast<uint32_t>((x >> p0) & (dm >> p0));
         uint32_t d = 0u;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          if (i < nb) d |= ((x >> pos[i]) & 1u) << i;
+          if (i < nb) d |= static_cast<uint32_t>((x >> pos[i]) & 1u) << i;
         return d;
       };
       for (int d = lane; d < kBins / 2; d += 32) cw[d] = 0u;
@@ -1237,10 +1238,10 @@ struct Finisher {
   // ascending) with a stable LSD radix sort of a 16-bit permutation, then the
   // first m written. Used when buckets stay crowded with equal keys (values
   // on a coarse grid, such as fp8 or bf16), where counting ranks inside a
-  // bucket would be quadratic. The 8-bit digits are laid over the span of
-  // bits that differ between the sorted candidates in each half of C (the
-  // indices of a 64K row take two passes, keys on the fp8 grid one). Ends
-  // with a barrier.
+  // bucket would be quadratic. The 8-bit digits are laid over the bits of C
+  // that differ between the sorted candidates, across both halves (a 128K
+  // row's 17 index bits and a bf16 grid's nine key bits take four passes).
+  // Ends with a barrier.
   __device__ __noinline__ static void finish_sorted(int n, int m, int k, uint32_t kmax, uint64_t cut, int64_t row,
                                                     const Params p, int fid) {
     Smem& s = cta_smem();
@@ -1302,11 +1303,9 @@ struct Finisher {
       vhi = a0 & ~a1;
       vlo = b0 & ~b1;
     }
-    for (int half = 0; half < 2; ++half) {
-      const uint32_t vary = half ? vhi : vlo;
-      if (vary == 0u) continue;  // the same in every candidate: its passes would be the identity
-      radix_passes(s, ns, kmax, half, vary, pa, pb, fid);
-    }
+    // one digit sequence over the varying bits of the whole composite (a digit
+    // may take the index's last bits and the key's first)
+    radix_passes(s, ns, kmax, (static_cast<uint64_t>(vhi) << 32) | vlo, pa, pb, fid);
     const int a = k >= 4 ? (3 * k) / 4 - 1 : 0;
     if (fid == 0) {
       if (m == k) s.rec[0] = cand_key(s)[pa[k - 1]];
