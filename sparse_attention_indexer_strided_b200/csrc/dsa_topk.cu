@@ -42,7 +42,8 @@ static std::mutex g_dev_mu;
 template <class T>
 static bool set_kernel_attributes() {
   const int smem = static_cast<int>(sizeof(rows::Smem));
-  if (cudaFuncSetAttribute(topk_rows_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+  if (cudaFuncSetAttribute(topk_rows_kernel<T, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      cudaFuncSetAttribute(topk_rows_kernel<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
       cudaFuncSetAttribute(topk_cluster_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     cudaGetLastError();
     return false;
@@ -56,7 +57,8 @@ static bool set_kernel_attributes() {
 template <class T>
 static bool built_with_launch_regs() {
   cudaFuncAttributes a;
-  return cudaFuncGetAttributes(&a, topk_rows_kernel<T>) == cudaSuccess && a.numRegs == rows::kLaunchRegs &&
+  return cudaFuncGetAttributes(&a, topk_rows_kernel<T, false>) == cudaSuccess && a.numRegs == rows::kLaunchRegs &&
+         cudaFuncGetAttributes(&a, topk_rows_kernel<T, true>) == cudaSuccess && a.numRegs == rows::kLaunchRegs &&
          cudaFuncGetAttributes(&a, topk_cluster_kernel<T>) == cudaSuccess && a.numRegs == rows::kLaunchRegs;
 }
 
@@ -72,7 +74,7 @@ static int device_setup(int dev, DeviceInfo* out) {
     // the library carries sm_100a code only, which runs on compute capability
     // 10.0 alone; the attribute query fails when no image loads on this device
     cudaFuncAttributes fa;
-    if (p.major != 10 || p.minor != 0 || cudaFuncGetAttributes(&fa, topk_rows_kernel<float>) != cudaSuccess) {
+    if (p.major != 10 || p.minor != 0 || cudaFuncGetAttributes(&fa, topk_rows_kernel<float, false>) != cudaSuccess) {
       cudaGetLastError();
       return DSA_ERR_NO_DEVICE;
     }
@@ -177,7 +179,11 @@ static int current_device(DeviceInfo* info) {
 
 template <class T>
 static cudaError_t launch_as(const cudaLaunchConfig_t& cfg, const rows::Params& p, bool clustered) {
-  return clustered ? cudaLaunchKernelEx(&cfg, topk_cluster_kernel<T>, p) : cudaLaunchKernelEx(&cfg, topk_rows_kernel<T>, p);
+  if (clustered) return cudaLaunchKernelEx(&cfg, topk_cluster_kernel<T>, p);
+  // rows that always fit one stage take the kernel instance that copies a
+  // stage with no threshold whole
+  if (p.row_stride <= rows::kShortStride) return cudaLaunchKernelEx(&cfg, topk_rows_kernel<T, true>, p);
+  return cudaLaunchKernelEx(&cfg, topk_rows_kernel<T, false>, p);
 }
 
 static int launch(const DeviceInfo& d, int32_t dtype, const rows::Params& p, cudaStream_t stream) {

@@ -88,6 +88,7 @@ constexpr int kWarpElems = 32 * kVals;                  // 1024 per warp and sta
 constexpr int kStageElems = kFilterWarps * kWarpElems;  // 8192
 constexpr int kRingBytes = 3 * 32768;                   // 96 KB ring
 constexpr int kMaxStages = 6;
+constexpr int64_t kShortStride = 8192 - 8;                // rows of at most this many elements are one stage
 constexpr int kFiltCap = 8192;                          // candidate buffer entries
 constexpr int kTrigger = kFiltCap / 2;                  // compact after a stage that leaves more
 constexpr int kHandCap = 4096;                          // handed-over (or gathered) candidates, at most
@@ -973,6 +974,39 @@ __device__ __forceinline__ void stream_item(Smem& s, Filter& f, RingPos& rp, con
   bar_filter();  // every append is visible
 }
 
+// An item of one stage with no threshold yet (a short row): every value in
+// [0, L) is a candidate, so the stage is copied into the candidate buffer in
+// index order, coalesced, with no pass masks or survivor exchange. Out of
+// line and outside the stage loop, so the streaming loop's code is untouched.
+struct OpenItem {
+  RingPos rp;    // the ring position after the stage
+  uint32_t cnt;  // candidates taken (0 if the stage's wait gave up)
+};
+
+template <class T>
+__device__ __noinline__ OpenItem stream_open(RingPos rp, int64_t j0, int32_t L, uint32_t base, int tid) {
+  Smem& s = cta_smem();
+  constexpr int kStages = stages_of<T>();
+  const int lane = tid & 31;
+  const bool ok = mbar_wait(&s.full[rp.slot], rp.phase, &s.wait);
+  const T* ring = reinterpret_cast<const T*>(s.ring) + rp.slot * kStageElems - j0;  // ring[e]: item index e
+  const int n = ok ? L : 0;
+  for (int e = tid; e < n; e += kFilterThreads) {
+    s.fkey[e] = to_key(Elem<T>::f(ring[e]));
+    s.fidx[e] = base + static_cast<uint32_t>(e);
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&s.empty[rp.slot]);
+  rp.par ^= 1u;
+  if (++rp.slot == kStages) {
+    rp.slot = 0;
+    rp.phase ^= 1u;
+  }
+  if (tid == 0) s.abort_seen = *reinterpret_cast<volatile uint32_t*>(&s.wait.abort);
+  bar_filter();  // every append is visible
+  return OpenItem{rp, static_cast<uint32_t>(n)};
+}
+
 // ---------------------------------------------------------- finisher
 // Ranks candidates hkey/hidx [0, n) by the composite C = (kmax - key) << 32 |
 // index (ascending C = key descending, index ascending; all C distinct) and
@@ -1572,7 +1606,10 @@ __device__ __noinline__ void joint_finish(const Params p, int tid) {
 
 
 
-template <class T>
+// kShort: the launch's row stride fits one stage (every row is one item of
+// one stage), and rows with no threshold take the stage whole (stream_open).
+// A separate kernel instance, so longer rows run unchanged code.
+template <class T, bool kShort>
 __device__ void filter_loop(Smem& s, const Params& p, int tid) {
   const int lane = tid & 31;
   const T* logits = static_cast<const T*>(p.logits);
@@ -1615,7 +1652,14 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
     f.compacted = false;
     f.strict = false;
     f.bounded = false;
-    stream_item<T>(s, f, rp, sp, L, 0u, m, tid);
+    if (kShort && sp.nst == 1 && !spec) {
+      const OpenItem o = stream_open<T>(rp, sp.j0, L, 0u, tid);
+      rp = o.rp;
+      f.cnt = o.cnt;
+      tighten(f, m);
+    } else {
+      stream_item<T>(s, f, rp, sp, L, 0u, m, tid);
+    }
     const bool reread = spec && !f.compacted && f.cnt < static_cast<uint32_t>(m) && !s.abort_seen;
     if (reread) {
       if (tid == 0) atomicOr(&g_status, kStatusReread);
@@ -2089,9 +2133,9 @@ __device__ __forceinline__ void init_cta(Smem& s) {
 }  // namespace rows
 
 // Many rows: grid = min(num_rows, SMs), one CTA per SM, rows strided by the
-// grid, 512 threads. (A kernel of its own, apart from the cluster mode, so
+// grid, 512 threads. kShort: every row fits one stage (see filter_loop). (A kernel of its own, apart from the cluster mode, so
 // that each gets its own register allocation.)
-template <class T>
+template <class T, bool kShort>
 __global__ void __launch_bounds__(rows::kThreads) topk_rows_kernel(const rows::Params p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   rows::Smem& s = *reinterpret_cast<rows::Smem*>(smem_raw);
@@ -2106,7 +2150,7 @@ __global__ void __launch_bounds__(rows::kThreads) topk_rows_kernel(const rows::P
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(rows::kOtherRegs) : "memory");
   }
   if (warp < rows::kFilterWarps) {
-    rows::filter_loop<T>(s, p, tid);
+    rows::filter_loop<T, kShort>(s, p, tid);
   } else if (warp < rows::kProducerWarp) {
     rows::finish_loop<T>(s, p, tid - rows::kFilterThreads);
   } else if (warp == rows::kProducerWarp && lane == 0) {

@@ -178,6 +178,34 @@ def test_cluster_rows_mostly_neg_inf(oracle_mod, dsa, k):
     assert_parity(oracle_mod, dsa, x, L, k)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("base_offset", [0, 3])
+def test_short_rows_kernel(oracle_mod, dsa, dtype, base_offset):
+    """Row strides that fit one stage take their own kernel instance, where a
+    row with no threshold is copied whole: many rows per CTA (later rows carry
+    thresholds), lengths past the 4096-entry handover (a compaction follows
+    the copy), ties, special values, an unaligned base."""
+    import torch
+    rng = np.random.default_rng(3400 + base_offset + (dtype == "bf16"))
+    rows, stride, k = 700, 8000, 2048
+    L = rng.integers(0, stride + 1, size=rows).astype(np.int32)
+    L[:6] = [0, 1, 2048, 4096, 4097, stride]
+    x = rng.standard_normal((rows, stride)).astype(np.float32)
+    x[1::4] = np.round(x[1::4] * 4) / 4
+    x[2, :50] = np.nan
+    x[3, 100:200] = np.inf
+    t = torch.from_numpy(x)
+    if dtype == "bf16":
+        t = t.to(torch.bfloat16)
+    buf = torch.full((base_offset + rows * stride + 8,), float("inf"), dtype=t.dtype)
+    buf[base_offset:base_offset + rows * stride] = t.reshape(-1)
+    d = buf.cuda()[base_offset:base_offset + rows * stride].view(rows, stride)
+    got = dsa.dsa_topk(d, torch.from_numpy(L).cuda(), k).cpu().numpy()
+    exp = oracle_mod.topk(t.float().numpy(), L, k)
+    np.testing.assert_array_equal(got, exp)
+    assert dsa.device_status() & dsa.STATUS_ERRORS == 0
+
+
 # --------------------------------------------------------- layout and poison
 @pytest.mark.parametrize("extra,offset", [(0, 0), (1, 0), (2, 1), (3, 3), (5, 2), (256, 0)])
 def test_unaligned_strides_and_bases(oracle_mod, dsa, extra, offset):
