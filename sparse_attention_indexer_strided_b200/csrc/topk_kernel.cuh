@@ -792,7 +792,7 @@ __device__ __forceinline__ Filter refilter_from_global(Smem& s, Filter f, RowSpa
 // Counters live in fidx, unused until the item streams. Two plain-atomic
 // passes instead of a radix select's three or four rounds with their
 // barriers.
-__device__ __forceinline__ uint32_t sample_kth(Smem& s, uint32_t need, uint32_t lo, uint32_t hi, int tid) {
+__device__ __forceinline__ uint32_t sample_kth(Smem& s, int nvals, uint32_t need, uint32_t lo, uint32_t hi, int tid) {
   constexpr int kBits = 10, kBins = 1 << kBits, kPer = kBins / kFilterThreads;  // 4 bins per thread
   const int w = tid >> 5, lane = tid & 31;
   uint32_t* hist = s.fidx;
@@ -806,7 +806,7 @@ __device__ __forceinline__ uint32_t sample_kth(Smem& s, uint32_t need, uint32_t 
 #pragma unroll
     for (int i = 0; i < kPer / 4; ++i) h4[i] = make_uint4(0u, 0u, 0u, 0u);
     bar_filter();
-    for (int e = tid; e < kSampleVals; e += kFilterThreads) {
+    for (int e = tid; e < nvals; e += kFilterThreads) {
       const uint32_t x = s.fkey[e];
       if (x >= base && x <= top) atomicAdd(&hist[(x - base) >> sh], 1u);
     }
@@ -856,7 +856,7 @@ __device__ __forceinline__ uint32_t sample_kth(Smem& s, uint32_t need, uint32_t 
   // grid's level, so that the filter's strict bound can later exclude its
   // further copies), with as many keys at or above it as the bin's edge
   uint32_t mn = 0xFFFFFFFFu;
-  for (int e = tid; e < kSampleVals; e += kFilterThreads) {
+  for (int e = tid; e < nvals; e += kFilterThreads) {
     const uint32_t x = s.fkey[e];
     if (x >= base && x <= top) mn = min(mn, x);
   }
@@ -874,8 +874,9 @@ __device__ __forceinline__ uint32_t sample_kth(Smem& s, uint32_t need, uint32_t 
 // the sample's count above m: a re-read is rare, and a looser margin costs
 // more in candidate writes and compactions than it saves. Returns -inf when
 // the sample gives none.
-template <class T>
+template <class T, int kRunsPerWarp = kSampleRunsPerWarp>
 __device__ __noinline__ float sample_threshold(const T* row, int64_t L, int m, int tid) {
+  constexpr int kChunks = kFilterWarps * kRunsPerWarp, kVals = kChunks * 128;
   Smem& s = cta_smem();
   const int w = tid >> 5, lane = tid & 31;
   const uintptr_t a = reinterpret_cast<uintptr_t>(row);
@@ -884,9 +885,9 @@ __device__ __noinline__ float sample_threshold(const T* row, int64_t L, int m, i
   const int64_t span = L - j0;                                      // elements from the aligned base to the end
   uint32_t mn = 0xFFFFFFFFu, mx = 0u;
 #pragma unroll
-  for (int q = 0; q < kSampleRunsPerWarp; ++q) {
-    const int64_t c = w * kSampleRunsPerWarp + q;
-    const int64_t b = ((span - 128) * c / (kSampleChunks - 1)) & ~static_cast<int64_t>(3);
+  for (int q = 0; q < kRunsPerWarp; ++q) {
+    const int64_t c = w * kRunsPerWarp + q;
+    const int64_t b = ((span - 128) * c / (kChunks - 1)) & ~static_cast<int64_t>(3);
     float xv[4];
     Elem<T>::four_ldg(reinterpret_cast<const T*>(as) + b + 4 * lane, xv);
 #pragma unroll
@@ -907,9 +908,9 @@ __device__ __noinline__ float sample_threshold(const T* row, int64_t L, int m, i
   bar_filter();
   mn = __reduce_min_sync(kFull, lane < kFilterWarps ? s.fred[0][lane] : 0xFFFFFFFFu);
   mx = __reduce_max_sync(kFull, lane < kFilterWarps ? s.fred[1][lane] : 0u);
-  const double share = static_cast<double>(kSampleVals) * m / static_cast<double>(L);
-  const uint32_t need = min(static_cast<uint32_t>(kSampleVals - 8), static_cast<uint32_t>(1.25 * share) + 12u);
-  const uint32_t T0 = sample_kth(s, need, mn, mx, tid);
+  const double share = static_cast<double>(kVals) * m / static_cast<double>(L);
+  const uint32_t need = min(static_cast<uint32_t>(kVals - 8), static_cast<uint32_t>(1.25 * share) + 12u);
+  const uint32_t T0 = sample_kth(s, kVals, need, mn, mx, tid);
   bar_filter();  // fkey, fidx, fred and bc are free again
   return (T0 == 0u || T0 >= kInfKey) ? __int_as_float(0xff800000) : from_key(T0);
 }
@@ -2061,7 +2062,9 @@ __device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid
   f.t = __int_as_float(0xff800000);
   bool spec = false;
   if (Lc >= kSampleMinLen && m_r > 0) {
-    const float ts = sample_threshold(rowp + it.c0, Lc, static_cast<int>(m_r), tid);
+    // a chunk samples 1024 values (one run per filter warp): the select's
+    // rounds cost less, and the threshold only bounds this rank's part
+    const float ts = sample_threshold<T, 1>(rowp + it.c0, Lc, static_cast<int>(m_r), tid);
     if (ts > __int_as_float(0xff800000)) {
       spec = true;
       f.t = ts;
@@ -2092,6 +2095,7 @@ __device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid
   }
   uint32_t total = cluster_merge(f.cnt, it.m, !ok, open, it.rank, it.ncta, tid);
   if (total == kMergeRetry) {  // the same on every rank of the cluster
+    if (tid == 0) atomicOr(&g_status, kStatusReread);
     f = refilter_from_global<T>(s, f, sp, Lc, static_cast<uint32_t>(it.c0), static_cast<int>(m_r), tid);
     if (f.cnt > static_cast<uint32_t>(kHandCap)) compact_any(s, f, static_cast<int>(m_r), tid);
     total = cluster_merge(f.cnt, it.m, !ok, false, it.rank, it.ncta, tid);

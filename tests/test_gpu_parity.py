@@ -329,7 +329,8 @@ def test_few_levels_many_rows(oracle_mod, dsa):
     assert_parity(oracle_mod, dsa, x, L, 100)
 
 
-SAMPLE_RUNS = 32    # a first threshold is sampled from 32 runs of 128 values
+SAMPLE_RUNS = 32    # a row's first threshold is sampled from 32 runs of 128 values
+CLUSTER_SAMPLE_RUNS = 8  # a cluster rank's from 8 (one per filter warp)
 CHUNK_ALIGN = 8     # a cluster rank's chunk is rounded up to a multiple of 8 elements
 
 
@@ -391,7 +392,7 @@ def test_sampled_threshold_fallback_cluster(oracle_mod, dsa):
     x = (rng.standard_normal((rows, stride)) * 0.01).astype(np.float32)
     for r in range(ranks):
         c0, c1 = min(L, r * chunk), min(L, r * chunk + chunk)
-        for b in _sample_runs(c1 - c0, SAMPLE_RUNS):
+        for b in _sample_runs(c1 - c0, CLUSTER_SAMPLE_RUNS):
             x[:, c0 + b:c0 + b + 128] = 100.0 + rng.random((rows, 128), dtype=np.float32)
     Ls = np.full(rows, L, np.int32)
     dsa.device_status(clear=True)
