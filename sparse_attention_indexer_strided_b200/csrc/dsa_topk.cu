@@ -26,9 +26,6 @@ namespace dsa {
 
 struct DeviceInfo {
   int sms = 0;
-  // every kernel instance was built with exactly rows::kLaunchRegs registers
-  // per thread, so the many-row register split balances (see kFilterRegs)
-  uint32_t regsplit = 0;
   // CTAs of a cluster launch of size 2, 4, 8, 16 that can be resident at once
   // (index log2 of the size; 0: that size does not launch on this device)
   int cluster_ctas[5] = {0, 0, 0, 0, 0};
@@ -53,15 +50,6 @@ static bool set_kernel_attributes() {
   return true;
 }
 
-// The register split needs exactly rows::kLaunchRegs registers per thread.
-template <class T>
-static bool built_with_launch_regs() {
-  cudaFuncAttributes a;
-  return cudaFuncGetAttributes(&a, topk_rows_kernel<T, false>) == cudaSuccess && a.numRegs == rows::kLaunchRegs &&
-         cudaFuncGetAttributes(&a, topk_rows_kernel<T, true>) == cudaSuccess && a.numRegs == rows::kLaunchRegs &&
-         cudaFuncGetAttributes(&a, topk_cluster_kernel<T>) == cudaSuccess && a.numRegs == rows::kLaunchRegs;
-}
-
 static int device_setup(int dev, DeviceInfo* out) {
   std::lock_guard<std::mutex> lock(g_dev_mu);
   DeviceInfo& d = g_dev[dev];
@@ -79,12 +67,6 @@ static int device_setup(int dev, DeviceInfo* out) {
       return DSA_ERR_NO_DEVICE;
     }
     d.sms = p.multiProcessorCount;
-    {
-      const bool ok = built_with_launch_regs<float>() && built_with_launch_regs<__nv_bfloat16>() &&
-                      built_with_launch_regs<__half>();
-      cudaGetLastError();
-      d.regsplit = ok ? 1u : 0u;
-    }
     if (!set_kernel_attributes<float>() || !set_kernel_attributes<__nv_bfloat16>() ||
         !set_kernel_attributes<__half>())
       return DSA_ERR_CONFIG;
@@ -229,7 +211,7 @@ static int run(const void* logits, int32_t dtype, int64_t row_stride, const int3
   DeviceInfo d;
   rc = current_device(&d);
   if (rc != DSA_OK) return rc;
-  const rows::Params p{logits, row_stride, lengths, num_rows, k, flags, table, table ? table_stride : 0, out, d.regsplit};
+  const rows::Params p{logits, row_stride, lengths, num_rows, k, flags, table, table ? table_stride : 0, out};
   return launch(d, dtype, p, stream);
 }
 
@@ -263,7 +245,7 @@ DSA_EXPORT int dsa_topk_host(const float* h_logits, int64_t row_stride, const in
     cudaGetLastError();
     return DSA_ERR_LAUNCH;
   }
-  const dsa::rows::Params p{d_logits, row_stride, d_lengths, num_rows, k, 0u, nullptr, 0, d_out, d.regsplit};
+  const dsa::rows::Params p{d_logits, row_stride, d_lengths, num_rows, k, 0u, nullptr, 0, d_out};
   rc = dsa::launch(d, DSA_DTYPE_F32, p, stream);
   if (rc != DSA_OK) return rc;
   if (cudaMemcpyAsync(h_out, d_out, static_cast<size_t>(num_rows) * k * sizeof(int32_t), cudaMemcpyDeviceToHost,

@@ -70,18 +70,6 @@ constexpr int kProducerWarp = kFilterWarps + kFinishWarps;
 constexpr int kThreads = 16 * 32;                       // 512: many-row mode (4 warpgroups; warp 15 idle)
 constexpr int kClusterWarp = kFilterWarps;              // cluster mode: the producer warp
 constexpr int kClusterThreads = 12 * 32;                // 384: cluster mode (3 warpgroups; warps 9-11 only mirror barriers)
-// Many-row mode moves registers between warpgroups (setmaxnreg): the filter
-// warpgroups take kFilterRegs per thread, the finisher / producer warpgroups
-// give up to kOtherRegs. The block is launched with 128 per thread (512 x 128
-// = the whole register file), and 2 x 160 + 2 x 96 = 4 x 128, so the split is
-// exactly the launch allocation; the host enables it only after checking that
-// every kernel instance was built with 128 registers per thread.
-// Cluster mode does the same with three warpgroups: 2 x 160 + 64 = 3 x 128.
-constexpr int kLaunchRegs = 128, kFilterRegs = 160, kOtherRegs = 96, kMirrorRegs = 64;
-static_assert(2 * kFilterRegs + 2 * kOtherRegs == 4 * kLaunchRegs && kThreads * kLaunchRegs == 65536,
-              "the register split must equal the launch allocation");
-static_assert(2 * kFilterRegs + kMirrorRegs == 3 * kLaunchRegs && kClusterThreads == 3 * 128,
-              "the cluster-mode register split must equal the launch allocation");
 constexpr int kGroups = 8;                              // groups of 4 values per lane and stage
 constexpr int kVals = 4 * kGroups;                      // 32 values per lane and stage
 constexpr int kWarpElems = 32 * kVals;                  // 1024 per warp and stage
@@ -127,7 +115,6 @@ struct Params {
   const int32_t* table;  // optional index table: out = table[row * table_stride + idx]
   int64_t table_stride;
   int32_t* out;
-  uint32_t regsplit;  // many-row mode: move registers between warpgroups (see kFilterRegs)
 };
 
 struct __align__(128) Smem {
@@ -1009,6 +996,11 @@ __device__ __noinline__ OpenItem stream_open(RingPos rp, int64_t j0, int32_t L, 
 }
 
 // ---------------------------------------------------------- finisher
+// Bounds on a candidate set known before its ranking starts.
+struct KeyBounds {
+  uint32_t kmin, kmax, imax;
+};
+
 // Ranks candidates hkey/hidx [0, n) by the composite C = (kmax - key) << 32 |
 // index (ascending C = key descending, index ascending; all C distinct) and
 // writes the first m to the output row. Buckets are 12-bit slices of C: count,
@@ -1361,38 +1353,49 @@ struct Finisher {
   // `alone`: nothing else runs on the SM meanwhile (a CTA's last row, a
   // cluster's leader).
   // (Inlined into the finisher warps' loop; a call there cost a few percent.)
+  // kb: NULL, or bounds the caller already holds (kmin <= every key <= kmax,
+  // every index <= imax); then the pass that finds them is skipped and the
+  // value grid is taken as unknown (finer passes before a sort, never a wrong
+  // rank: every choice below only picks among exact methods)
   __device__ __forceinline__ static void finish(Smem& s, int n, int m, int k, int64_t row, const Params& p, int fid,
-                                                bool alone) {
+                                                bool alone, const KeyBounds* kb = nullptr) {
     const int fw = fid >> 5, lane = fid & 31;
     int32_t* o = p.out + row * static_cast<int64_t>(k);
     for (int q = m + fid; q < k; q += NT) o[q] = -1;
     if (n <= 0) return;
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, imax = 0u, kdiff = 0u;
-    const uint32_t key0 = cand_key(s)[0];
-    for (int e = fid; e < n; e += NT) {
-      const uint32_t key = cand_key(s)[e];
-      kmin = min(kmin, key);
-      kmax = max(kmax, key);
-      kdiff |= key ^ key0;
-      imax = max(imax, cand_idx(s)[e]);
-    }
-    kmin = __reduce_min_sync(kFull, kmin);
-    kmax = __reduce_max_sync(kFull, kmax);
-    imax = __reduce_max_sync(kFull, imax);
-    kdiff = __reduce_or_sync(kFull, kdiff);
-    if (lane == 0) {
-      s.nred[0][fw] = kmin;
-      s.nred[1][fw] = kmax;
-      s.nred[2][fw] = imax;
-      s.nred[3][fw] = kdiff;
-    }
-    bar();
+    if (kb != nullptr) {
+      kmin = kb->kmin;
+      kmax = kb->kmax;
+      imax = kb->imax;
+      kdiff = kmin == kmax ? 0u : 1u;  // equal bounds: one key; else grid 0
+    } else {
+      const uint32_t key0 = cand_key(s)[0];
+      for (int e = fid; e < n; e += NT) {
+        const uint32_t key = cand_key(s)[e];
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
+        kdiff |= key ^ key0;
+        imax = max(imax, cand_idx(s)[e]);
+      }
+      kmin = __reduce_min_sync(kFull, kmin);
+      kmax = __reduce_max_sync(kFull, kmax);
+      imax = __reduce_max_sync(kFull, imax);
+      kdiff = __reduce_or_sync(kFull, kdiff);
+      if (lane == 0) {
+        s.nred[0][fw] = kmin;
+        s.nred[1][fw] = kmax;
+        s.nred[2][fw] = imax;
+        s.nred[3][fw] = kdiff;
+      }
+      bar();
 #pragma unroll
-    for (int ww = 0; ww < kWarps; ++ww) {
-      kmin = min(kmin, s.nred[0][ww]);
-      kmax = max(kmax, s.nred[1][ww]);
-      imax = max(imax, s.nred[2][ww]);
-      kdiff |= s.nred[3][ww];
+      for (int ww = 0; ww < kWarps; ++ww) {
+        kmin = min(kmin, s.nred[0][ww]);
+        kmax = max(kmax, s.nred[1][ww]);
+        imax = max(imax, s.nred[2][ww]);
+        kdiff |= s.nred[3][ww];
+      }
     }
     // every two keys differ by a multiple of 2^grid (keys on a value grid,
     // such as fp8 or bf16 values, have zero low bits): buckets no wider than
@@ -1943,6 +1946,7 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
   if (tid == 0) {
     s.pub[4] = g_r;
     s.pub[5] = exact ? q_r : 0u;
+    s.bc[5] = lo;  // every key copied to the leader is >= lo (bc[4] still holds the max)
   }
   cluster_barrier();
   ++nbar;
@@ -2105,7 +2109,8 @@ __device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid
     for (int q = tid; q < k; q += kFilterThreads) p.out[it.row * static_cast<int64_t>(k) + q] = -1;
     return;
   }
-  LeaderFinisher::finish(s, static_cast<int>(total), static_cast<int>(it.m), k, it.row, p, tid, true);
+  const KeyBounds kb{s.bc[5], s.bc[4], static_cast<uint32_t>(it.L - 1)};
+  LeaderFinisher::finish(s, static_cast<int>(total), static_cast<int>(it.m), k, it.row, p, tid, true, &kb);
 }
 
 // Shared state of a fresh CTA (thread 0; a barrier follows).
@@ -2147,12 +2152,6 @@ __global__ void __launch_bounds__(rows::kThreads) topk_rows_kernel(const rows::P
   if (tid == 0) rows::init_cta(s);
   __syncthreads();
   pdl_enter();  // every thread: inputs and outputs are touched only after this
-  if (p.regsplit) {  // whole warpgroups: warps 0-7 filter; the rest finisher / producer
-    if (warp < rows::kFilterWarps)
-      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(rows::kFilterRegs) : "memory");
-    else
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(rows::kOtherRegs) : "memory");
-  }
   if (warp < rows::kFilterWarps) {
     rows::filter_loop<T, kShort>(s, p, tid);
   } else if (warp < rows::kProducerWarp) {
@@ -2171,12 +2170,6 @@ __global__ void __launch_bounds__(rows::kThreads) topk_cluster_kernel(const rows
   if (tid == 0) rows::init_cta(s);
   __syncthreads();
   pdl_enter();  // every thread: inputs and outputs are touched only after this
-  if (p.regsplit) {  // whole warpgroups: warps 0-7 filter; warps 8-11 producer / mirror
-    if (warp < rows::kFilterWarps)
-      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(rows::kFilterRegs) : "memory");
-    else
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(rows::kMirrorRegs) : "memory");
-  }
   if (warp < rows::kFilterWarps)
     rows::cluster_filter<T>(s, p, tid);
   else
