@@ -134,6 +134,7 @@ struct __align__(128) Smem {
   uint32_t small[32];
   uint32_t rec[2];  // finisher: keys at ranks k-1 and 3k/4-1
   uint32_t pub[8];  // cluster mode: published to the other ranks
+  uint32_t spub[4];  // cluster mode: [0..2] this rank's sample count and key bounds, read by the others; [3] the merge's key-difference bits
   // handover (filter -> finisher)
   int64_t h_row, h_len;
   int32_t h_n, h_m;
@@ -861,16 +862,20 @@ __device__ __forceinline__ uint32_t sample_kth(Smem& s, int nvals, uint32_t need
 // the sample's count above m: a re-read is rare, and a looser margin costs
 // more in candidate writes and compactions than it saves. Returns -inf when
 // the sample gives none.
-template <class T, int kRunsPerWarp = kSampleRunsPerWarp>
-__device__ __noinline__ float sample_threshold(const T* row, int64_t L, int m, int tid) {
-  constexpr int kChunks = kFilterWarps * kRunsPerWarp, kVals = kChunks * 128;
-  Smem& s = cta_smem();
+// Loads kFilterWarps * kRunsPerWarp evenly spaced runs of 128 values (aligned
+// 16-byte blocks inside the item) into fkey as keys, 0 for a position outside
+// [0, L) (below every key), and returns their smallest and largest key in
+// every filter thread.
+template <class T, int kRunsPerWarp>
+__device__ __forceinline__ void sample_keys(Smem& s, const T* row, int64_t L, int tid, uint32_t& mn, uint32_t& mx) {
+  constexpr int kChunks = kFilterWarps * kRunsPerWarp;
   const int w = tid >> 5, lane = tid & 31;
   const uintptr_t a = reinterpret_cast<uintptr_t>(row);
   const uintptr_t as = a & ~static_cast<uintptr_t>(15);
   const int64_t j0 = -static_cast<int64_t>((a - as) / sizeof(T));  // item index of the aligned base
   const int64_t span = L - j0;                                      // elements from the aligned base to the end
-  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+  mn = 0xFFFFFFFFu;
+  mx = 0u;
 #pragma unroll
   for (int q = 0; q < kRunsPerWarp; ++q) {
     const int64_t c = w * kRunsPerWarp + q;
@@ -895,9 +900,24 @@ __device__ __noinline__ float sample_threshold(const T* row, int64_t L, int m, i
   bar_filter();
   mn = __reduce_min_sync(kFull, lane < kFilterWarps ? s.fred[0][lane] : 0xFFFFFFFFu);
   mx = __reduce_max_sync(kFull, lane < kFilterWarps ? s.fred[1][lane] : 0u);
-  const double share = static_cast<double>(kVals) * m / static_cast<double>(L);
-  const uint32_t need = min(static_cast<uint32_t>(kVals - 8), static_cast<uint32_t>(1.25 * share) + 12u);
-  const uint32_t T0 = sample_kth(s, kVals, need, mn, mx, tid);
+}
+
+// A threshold for an item with no estimate, from a sample of kSampleVals
+// values in kSampleChunks evenly spaced runs of 128 (aligned 16-byte blocks
+// inside the item): the value with as many sampled values above it as 1.25
+// times the share of m in the sample, plus 12. On a 128K-value row with k =
+// 2048 that lets about 2.9K values through, some three standard deviations of
+// the sample's count above m: a re-read is rare, and a looser margin costs
+// more in candidate writes and compactions than it saves. Returns -inf when
+// the sample gives none.
+template <class T>
+__device__ __noinline__ float sample_threshold(const T* row, int64_t L, int m, int tid) {
+  Smem& s = cta_smem();
+  uint32_t mn, mx;
+  sample_keys<T, kSampleRunsPerWarp>(s, row, L, tid, mn, mx);
+  const double share = static_cast<double>(kSampleVals) * m / static_cast<double>(L);
+  const uint32_t need = min(static_cast<uint32_t>(kSampleVals - 8), static_cast<uint32_t>(1.25 * share) + 12u);
+  const uint32_t T0 = sample_kth(s, kSampleVals, need, mn, mx, tid);
   bar_filter();  // fkey, fidx, fred and bc are free again
   return (T0 == 0u || T0 >= kInfKey) ? __int_as_float(0xff800000) : from_key(T0);
 }
@@ -996,9 +1016,11 @@ __device__ __noinline__ OpenItem stream_open(RingPos rp, int64_t j0, int32_t L, 
 }
 
 // ---------------------------------------------------------- finisher
-// Bounds on a candidate set known before its ranking starts.
+// Bounds on a candidate set known before its ranking starts: kmin <= every
+// key <= kmax, every index <= imax, and kdiff has every bit in which two of
+// the keys may differ.
 struct KeyBounds {
-  uint32_t kmin, kmax, imax;
+  uint32_t kmin, kmax, imax, kdiff;
 };
 
 // Ranks candidates hkey/hidx [0, n) by the composite C = (kmax - key) << 32 |
@@ -1353,10 +1375,9 @@ struct Finisher {
   // `alone`: nothing else runs on the SM meanwhile (a CTA's last row, a
   // cluster's leader).
   // (Inlined into the finisher warps' loop; a call there cost a few percent.)
-  // kb: NULL, or bounds the caller already holds (kmin <= every key <= kmax,
-  // every index <= imax); then the pass that finds them is skipped and the
-  // value grid is taken as unknown (finer passes before a sort, never a wrong
-  // rank: every choice below only picks among exact methods)
+  // kb: NULL, or bounds the caller already holds; then the pass that finds
+  // them is skipped (looser bounds than the pass would find only change which
+  // exact method is picked below)
   __device__ __forceinline__ static void finish(Smem& s, int n, int m, int k, int64_t row, const Params& p, int fid,
                                                 bool alone, const KeyBounds* kb = nullptr) {
     const int fw = fid >> 5, lane = fid & 31;
@@ -1368,7 +1389,7 @@ struct Finisher {
       kmin = kb->kmin;
       kmax = kb->kmax;
       imax = kb->imax;
-      kdiff = kmin == kmax ? 0u : 1u;  // equal bounds: one key; else grid 0
+      kdiff = kb->kdiff;
     } else {
       const uint32_t key0 = cand_key(s)[0];
       for (int e = fid; e < n; e += NT) {
@@ -1766,13 +1787,14 @@ __device__ void finish_loop(Smem& s, const Params& p, int fid) {
 }
 
 // ---------------------------------------------------------- producer
-// Issues one item's stages into the ring. Returns false when a wait gave up.
+// Issues stages [st0, st1) of an item into the ring. Returns false when a wait
+// gave up.
 template <class T>
-__device__ __forceinline__ bool produce_span(Smem& s, const RowSpan& sp, int& slot, uint32_t& phase, long long& gi,
-                                             long long skip, uint32_t& armed, uint32_t& arm_par) {
+__device__ __forceinline__ bool produce_stages(Smem& s, const RowSpan& sp, int st0, int st1, int& slot, uint32_t& phase,
+                                               long long& gi, long long skip, uint32_t& armed, uint32_t& arm_par) {
   constexpr int kStages = stages_of<T>();
   constexpr uint32_t kStageBytes = kStageElems * sizeof(T);
-  for (int st = 0; st < sp.nst; ++st, ++gi) {
+  for (int st = st0; st < st1; ++st, ++gi) {
     if (!mbar_wait_sleep(&s.empty[slot], phase ^ 1u, &s.wait)) return false;
     if (gi != skip) {
       const uint32_t bytes = st + 1 == sp.nst ? sp.last_bytes : kStageBytes;
@@ -1789,6 +1811,13 @@ __device__ __forceinline__ bool produce_span(Smem& s, const RowSpan& sp, int& sl
     }
   }
   return true;
+}
+
+// Issues one item's stages into the ring. Returns false when a wait gave up.
+template <class T>
+__device__ __forceinline__ bool produce_span(Smem& s, const RowSpan& sp, int& slot, uint32_t& phase, long long& gi,
+                                             long long skip, uint32_t& armed, uint32_t& arm_par) {
+  return produce_stages<T>(s, sp, 0, sp.nst, slot, phase, gi, skip, armed, arm_par);
 }
 
 // Before returning, on the normal path and after an abort alike, the producer
@@ -1814,30 +1843,145 @@ __device__ void produce_loop(Smem& s, const Params& p) {
 }
 
 // ---------------------------------------------------------- cluster mode
-// After streaming, rank `rank` holds n_r candidates in fkey/fidx, a superset
-// of its chunk's top min(m, chunk) (none if a wait gave up). The filter warps
-// of every rank run the merge; at the leader (rank 0) the survivors end in
-// hkey/hidx. Returns the number gathered there. The producer warp mirrors
-// every cluster barrier (s.final_bar tells it how many there are).
 constexpr uint32_t kMergeRetry = 0xFFFFFFFFu;
 constexpr int kMaxClusterSize = 16;  // the largest cluster the host plans
+constexpr int kSampleBars = 3;       // cluster barriers of cluster_threshold, on every path
 
-__device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool aborted, bool open, uint32_t rank,
+// Sum over the cluster's ranks of bin tid of the 256-bin histogram ph (the
+// same shared-memory offset in every rank). The remote loads are all issued
+// before any is summed: one at a time, each load's round trip would add up
+// across the cluster.
+__device__ __forceinline__ uint32_t cluster_bin_sum(const uint32_t* ph, uint32_t ncta, int tid) {
+  const uint32_t a = smem_addr(&ph[tid]);
+  uint32_t v[kMaxClusterSize];
+#pragma unroll
+  for (int r = 0; r < kMaxClusterSize; ++r) v[r] = static_cast<uint32_t>(r) < ncta ? dsmem_ld(dsmem_map(a, r)) : 0u;
+  uint32_t g = 0;
+#pragma unroll
+  for (int r = 0; r < kMaxClusterSize; ++r) g += v[r];
+  return g;
+}
+
+// One threshold for a whole cluster-split row, from every rank's sample: each
+// rank with a chunk of at least kSampleMinLen samples 1024 of its values (one
+// run of 128 per filter warp); the ranks publish their sample counts and key
+// bounds, then two cluster-wide 256-bin histogram rounds narrow the bin that
+// holds the need-th largest of all samples, need being the sample's share of
+// m with the margin of the single-row threshold (1.25 x + 12). Keys at or
+// above the final bin's lower edge number at least `need` among the samples;
+// on a row of 900K values with m = 1024 the threshold lets about 1.9K values
+// through in total, where a threshold from each rank's own sample must let
+// m-plus-margin through in every rank (a rank's chunk may hold the whole top
+// m). Every rank computes the same threshold from the same sums, which is
+// what lets the merge check it: if the ranks together hold at least m values
+// at or above it, those contain the row's top m.
+// Returns -inf when the samples give no threshold above -inf (or one at or
+// above +inf). Runs exactly kSampleBars cluster barriers on every path (the
+// producer warpgroup runs as many). The histograms go in the merge's slots of
+// bcnt, which the filter warps leave alone until the merge, whose first
+// cluster barrier every rank reaches only after it has read them.
+template <class T>
+__device__ __noinline__ float cluster_threshold(const T* chunk, int64_t Lc, int64_t L, uint32_t m, uint32_t ncta,
+                                                int tid) {
+  Smem& s = cta_smem();
+  const int w = tid >> 5, lane = tid & 31;
+  constexpr uint32_t kRankVals = kFilterWarps * 128;
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u, ns = 0u;
+  if (Lc >= kSampleMinLen) {
+    sample_keys<T, 1>(s, chunk, Lc, tid, mn, mx);
+    ns = kRankVals;
+  }
+  if (tid == 0) {
+    s.spub[0] = ns;
+    s.spub[1] = mn;
+    s.spub[2] = mx;
+  }
+  cluster_barrier();
+  if (w == 0) {
+    uint32_t n = 0, lo_r = 0xFFFFFFFFu, hi_r = 0u;
+    if (lane < static_cast<int>(ncta)) {
+      const uint32_t a = dsmem_map(smem_addr(&s.spub[0]), lane);
+      n = dsmem_ld(a);
+      lo_r = dsmem_ld(a + 4);
+      hi_r = dsmem_ld(a + 8);
+    }
+    n = __reduce_add_sync(kFull, n);
+    lo_r = __reduce_min_sync(kFull, lo_r);
+    hi_r = __reduce_max_sync(kFull, hi_r);
+    if (lane == 0) {
+      s.bc[2] = n;
+      s.bc[3] = lo_r;
+      s.bc[4] = hi_r;
+    }
+  }
+  bar_filter();
+  const uint32_t N = s.bc[2];
+  uint32_t lo = s.bc[3], hi = s.bc[4];
+  const double share = static_cast<double>(N) * m / static_cast<double>(L);
+  uint32_t need = N > 16u ? min(N - 8u, static_cast<uint32_t>(1.25 * share) + 12u) : 0u;
+  bool ok = need > 0u;  // the same in every rank (N, m and L are)
+  uint32_t* ghist = s.bcnt + 512;
+#pragma unroll 1
+  for (int round = 0; round < kSampleBars - 1; ++round) {
+    uint32_t* ph = s.bcnt + 256 * round;
+    const bool live = ok && lo != hi;
+    const int sh = live ? window_shift(lo, hi) : 0;
+    ph[tid] = 0u;  // kFilterThreads == 256
+    if (tid == 0) s.bc[0] = 0xFFFFFFFFu;
+    bar_filter();
+    if (live) digit_histogram(ph, static_cast<int>(ns), FKey{&s}, FAll{}, lo, hi, sh, tid);
+    cluster_barrier();
+    if (live) {
+      ghist[tid] = cluster_bin_sum(ph, ncta, tid);
+      bar_filter();
+      if (w == 0) find_bucket_warp0(ghist, need, s.bc, lane);
+      bar_filter();
+      const uint32_t b = s.bc[0];
+      if (b == 0xFFFFFFFFu) {  // the same sums in every rank: the same outcome
+        ok = false;
+      } else {
+        need -= s.bc[1];
+        narrow(lo, hi, sh, b);
+      }
+    }
+    bar_filter();  // bc and ghist are rewritten by the next round
+  }
+  return (ok && lo > to_key(__int_as_float(0xff800000)) && lo < kInfKey) ? from_key(lo) : __int_as_float(0xff800000);
+}
+
+// After streaming, rank `rank` holds n_r candidates in fkey/fidx (none if a
+// wait gave up): every value of its chunk at or above the row's threshold,
+// or, once the rank compacted, a superset of its chunk's top min(m, chunk).
+// The filter warps of every rank run the merge; at the leader (rank 0) the
+// survivors end in hkey/hidx. Returns the number gathered there, or
+// kMergeRetry when some rank's threshold was a guess (guessed) and the ranks
+// together hold fewer than m: then every rank takes its chunk again with no
+// threshold and merges once more. The producer warp mirrors every cluster
+// barrier (s.final_bar tells it how many there are).
+__device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool aborted, bool guessed, uint32_t rank,
                                                uint32_t ncta, int tid) {
   Smem& s = cta_smem();
   const int w = tid >> 5, lane = tid & 31;
   uint32_t nbar = s.merge_bars;
   uint32_t* phist = s.bcnt;        // [2][256], per rank, read by the others
   uint32_t* ghist = s.bcnt + 512;  // [256], cluster sums
-  // ---- phase 1: publish (count, min key, max key, gave up) of this rank
+  // ---- phase 1: publish (count, min key, max key, gave up, guessed, the
+  // bits in which a key differs from the max) of this rank
   uint32_t mn, mx;
   filter_minmax(s, static_cast<int>(n_r), FKey{&s}, FAll{}, mn, mx, tid);
+  uint32_t kd = 0u;
+  for (int e = tid; e < static_cast<int>(n_r); e += kFilterThreads) kd |= s.fkey[e] ^ mx;
+  kd = __reduce_or_sync(kFull, kd);
+  if (lane == 0) s.fred[2][w] = kd;
+  bar_filter();
+  kd = __reduce_or_sync(kFull, lane < kFilterWarps ? s.fred[2][lane] : 0u);
   if (tid == 0) {
+    s.pub[7] = kd;
     s.pub[0] = n_r;
     s.pub[1] = mn;
     s.pub[2] = mx;
     s.pub[3] = aborted ? 1u : 0u;
-    s.pub[6] = open ? 1u : 0u;
+    s.pub[6] = guessed ? 1u : 0u;
   }
   cluster_barrier();
   ++nbar;
@@ -1850,6 +1994,7 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
       hi_r = dsmem_ld(a + 8);
       ab = dsmem_ld(a + 12);
       op = dsmem_ld(a + 24);
+      kd = dsmem_ld(a + 28);
     }
     const bool full_rank = lane < static_cast<int>(ncta) && n >= m;
     const uint32_t N = __reduce_add_sync(kFull, n);
@@ -1859,16 +2004,20 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
     const uint32_t B = __reduce_max_sync(kFull, full_rank ? lo_r : 0u);
     const bool any_full = __ballot_sync(kFull, full_rank) != 0;
     const bool any_ab = __ballot_sync(kFull, ab != 0u) != 0;
-    const bool any_open = __ballot_sync(kFull, op != 0u) != 0;
+    const bool any_guess = __ballot_sync(kFull, op != 0u) != 0;
+    // bits in which two candidates of the cluster may differ (the leader's
+    // ranking detects a value grid from them)
+    const uint32_t kdall = __reduce_or_sync(kFull, n > 0u ? (kd | (hi_r ^ gmax)) : 0u);
     if (lane == 0) {
       s.bc[2] = N;
       s.bc[3] = any_full ? B : gmin;
       s.bc[4] = gmax;
       s.bc[5] = gmin;
+      s.spub[3] = kdall;  // read by the leader's ranking
       s.abort_any = any_ab ? 1u : 0u;
-      // fewer than m candidates, and some rank left out its -inf values: they
+      // fewer than m candidates under a guessed threshold: values below it
       // are needed, so every rank takes its chunk again with no threshold
-      s.merge_retry = (any_open && N < m && !any_ab) ? 1u : 0u;
+      s.merge_retry = (any_guess && N < m && !any_ab) ? 1u : 0u;
     }
   }
   bar_filter();
@@ -1886,8 +2035,12 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
   }
   uint32_t need = m;
   bool exact = false;
-  if (N <= static_cast<uint32_t>(kHandCap)) {
-    lo = gmin;  // everything fits at the leader
+  // Everything goes to the leader when it fits and holds little more than m;
+  // otherwise at least one round narrows it (with values on a coarse grid,
+  // usually to m plus one tied level: a leader ranking twice m tied
+  // candidates costs more than the round)
+  if (N <= static_cast<uint32_t>(kHandCap) && N <= m + (m >> 3)) {
+    lo = gmin;
   } else {
     // ---- phase 2: cluster-wide histogram rounds until the survivors fit
     int hp = 0;
@@ -1905,19 +2058,7 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
       digit_histogram(ph, static_cast<int>(n_r), FKey{&s}, FAll{}, lo, hi, sh, tid);
       cluster_barrier();
       ++nbar;
-      {
-        // every rank's count for this thread's bin: the remote loads are all
-        // issued before any is summed (one at a time, each load's round trip
-        // would add up across the cluster)
-        const uint32_t a = smem_addr(&ph[tid]);
-        uint32_t v[kMaxClusterSize];
-#pragma unroll
-        for (int r = 0; r < kMaxClusterSize; ++r) v[r] = static_cast<uint32_t>(r) < ncta ? dsmem_ld(dsmem_map(a, r)) : 0u;
-        uint32_t g = 0;
-#pragma unroll
-        for (int r = 0; r < kMaxClusterSize; ++r) g += v[r];
-        ghist[tid] = g;
-      }
+      ghist[tid] = cluster_bin_sum(ph, ncta, tid);  // every rank's count for this thread's bin
       bar_filter();
       if (w == 0) find_bucket_warp0(ghist, need, s.bc, lane);
       bar_filter();
@@ -2021,21 +2162,31 @@ __device__ __forceinline__ ClusterItem cluster_item(const Params& p) {
 }
 
 // Cluster mode, warps kClusterWarp.. (one warpgroup): lane 0 of the first
-// streams the chunk into the ring; then every warp of the group mirrors the
-// merge's cluster barriers (s.final_bar tells how many), leaving after the last.
+// streams the chunk into the ring. The ring's first fill waits for nothing,
+// so it is issued before the filter warps' sample exchange, whose
+// kSampleBars cluster barriers every warp of the group takes too; then the
+// rest of the chunk. Then every warp of the group mirrors the merge's
+// cluster barriers (s.final_bar tells how many), leaving after the last.
 template <class T>
 __device__ __noinline__ void cluster_mirror(const Params p, int tid) {
   Smem& s = cta_smem();
   const int w = tid >> 5, lane = tid & 31;
   const ClusterItem it = cluster_item(p);
   if (it.m == 0) return;  // the same for every CTA of the cluster: no merge, no barrier
-  if (w == kClusterWarp && lane == 0) {
-    const T* rowp = static_cast<const T*>(p.logits) + it.row * p.row_stride;
-    const RowSpan sp = row_span(rowp + it.c0, it.c1 - it.c0);
-    int slot = 0;
-    uint32_t phase = 0u, armed = 0u, arm_par = 0u;
-    long long gi = 0;
-    produce_span<T>(s, sp, slot, phase, gi, g_skip_stage, armed, arm_par);
+  const bool producer = w == kClusterWarp && lane == 0;
+  const T* rowp = static_cast<const T*>(p.logits) + it.row * p.row_stride;
+  const RowSpan sp = row_span(rowp + it.c0, it.c1 - it.c0);
+  const int first = min(sp.nst, stages_of<T>());
+  int slot = 0;
+  uint32_t phase = 0u, armed = 0u, arm_par = 0u;
+  long long gi = 0;
+  bool live = true;
+  if (producer) live = produce_stages<T>(s, sp, 0, first, slot, phase, gi, g_skip_stage, armed, arm_par);
+  __syncwarp();
+#pragma unroll 1
+  for (int i = 0; i < kSampleBars; ++i) cluster_barrier();
+  if (producer) {
+    if (live) produce_stages<T>(s, sp, first, sp.nst, slot, phase, gi, g_skip_stage, armed, arm_par);
     producer_drain(s, armed, arm_par);
   }
   __syncwarp();
@@ -2063,24 +2214,13 @@ __device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid
   const uint32_t m_r = min(it.m, static_cast<uint32_t>(Lc));
   Filter f;
   f.par = 0;
-  f.t = __int_as_float(0xff800000);
-  bool spec = false;
-  if (Lc >= kSampleMinLen && m_r > 0) {
-    // a chunk samples 1024 values (one run per filter warp): the select's
-    // rounds cost less, and the threshold only bounds this rank's part
-    const float ts = sample_threshold<T, 1>(rowp + it.c0, Lc, static_cast<int>(m_r), tid);
-    if (ts > __int_as_float(0xff800000)) {
-      spec = true;
-      f.t = ts;
-    }
-  }
-  // With no sampled threshold the rank keeps only values above -inf: a chunk
-  // of -inf (a row's padded tail) would otherwise fill the buffer with ties
-  // and cut them by index while the other ranks wait at the merge. The merge
-  // takes the chunks again with no threshold if the row turns out to hold
-  // fewer than m values above -inf.
-  const bool open = !spec;
-  if (open) f.t = __int_as_float(0xff7fffff);  // -FLT_MAX: keep x unless x < -FLT_MAX, i.e. x = -inf
+  // the row's threshold, the same in every rank (every rank takes part, a
+  // rank with a short chunk sampling nothing)
+  f.t = cluster_threshold<T>(rowp + it.c0, Lc, it.L, it.m, it.ncta, tid);
+  // With no threshold from the samples the rank keeps only values above -inf:
+  // a chunk of -inf (a row's padded tail) would otherwise fill the buffer with
+  // ties and cut them by index while the other ranks wait at the merge.
+  if (!(f.t > __int_as_float(0xff800000))) f.t = __int_as_float(0xff7fffff);  // -FLT_MAX: keep x unless x = -inf
   f.cnt = 0;
   f.compacted = false;
   f.strict = false;
@@ -2090,14 +2230,12 @@ __device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid
   const bool ok = !s.abort_seen;
   if (!ok) {
     f.cnt = 0;  // no candidates from this rank; it still takes part in the merge
-  } else {
-    if (spec && !f.compacted && f.cnt < m_r) {
-      if (tid == 0) atomicOr(&g_status, kStatusReread);
-      f = refilter_from_global<T>(s, f, sp, Lc, static_cast<uint32_t>(it.c0), static_cast<int>(m_r), tid);
-    }
-    if (f.cnt > static_cast<uint32_t>(kHandCap)) compact_any(s, f, static_cast<int>(m_r), tid);
+  } else if (f.cnt > static_cast<uint32_t>(kHandCap)) {
+    compact_any(s, f, static_cast<int>(m_r), tid);
   }
-  uint32_t total = cluster_merge(f.cnt, it.m, !ok, open, it.rank, it.ncta, tid);
+  // Either threshold is a guess: the merge checks that the ranks together
+  // hold at least m values, or has every rank take its chunk again with none.
+  uint32_t total = cluster_merge(f.cnt, it.m, !ok, true, it.rank, it.ncta, tid);
   if (total == kMergeRetry) {  // the same on every rank of the cluster
     if (tid == 0) atomicOr(&g_status, kStatusReread);
     f = refilter_from_global<T>(s, f, sp, Lc, static_cast<uint32_t>(it.c0), static_cast<int>(m_r), tid);
@@ -2109,7 +2247,7 @@ __device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid
     for (int q = tid; q < k; q += kFilterThreads) p.out[it.row * static_cast<int64_t>(k) + q] = -1;
     return;
   }
-  const KeyBounds kb{s.bc[5], s.bc[4], static_cast<uint32_t>(it.L - 1)};
+  const KeyBounds kb{s.bc[5], s.bc[4], static_cast<uint32_t>(it.L - 1), s.spub[3]};
   LeaderFinisher::finish(s, static_cast<int>(total), static_cast<int>(it.m), k, it.row, p, tid, true, &kb);
 }
 

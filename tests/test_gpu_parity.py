@@ -179,6 +179,33 @@ def test_cluster_rows_mostly_neg_inf(oracle_mod, dsa, k):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_cluster_threshold_shared_by_ranks(oracle_mod, dsa, dtype):
+    """Cluster ranks filter with one threshold drawn from every rank's sample.
+    Rows where it lies far from a rank's own share: values rising along the
+    row (the whole top k in the last chunk), 1000 large values placed between
+    two sample runs of one chunk, one chunk of shifted values on a coarse grid
+    (ties at the cut), and a plain row of another length."""
+    import torch
+    rng = np.random.default_rng(3500 + (dtype == "bf16"))
+    rows, stride, k = 4, 600000, 2048
+    L = np.array([stride, stride - 5, stride, 400001], np.int32)
+    x = rng.standard_normal((rows, stride)).astype(np.float32)
+    x[0] = np.sort(x[0])
+    x[1, 302000:303000] += 50.0  # inside one rank's chunk, clear of its sample runs
+    chunk = stride // 16
+    x[2, 5 * chunk:6 * chunk] = np.round(rng.standard_normal(chunk) * 4) / 4 + 3.0
+    t = torch.from_numpy(x)
+    if dtype == "bf16":
+        t = t.to(torch.bfloat16)
+    assert dsa.plan(rows, stride, k)[0] > 1
+    dsa.device_status(clear=True)
+    got = dsa.dsa_topk(t.cuda(), torch.from_numpy(L).cuda(), k).cpu().numpy()
+    exp = oracle_mod.topk(t.float().numpy(), L, k)
+    np.testing.assert_array_equal(got, exp)
+    assert dsa.device_status() & dsa.STATUS_ERRORS == 0
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("base_offset", [0, 3])
 def test_short_rows_kernel(oracle_mod, dsa, dtype, base_offset):
     """Row strides that fit one stage take their own kernel instance, where a
