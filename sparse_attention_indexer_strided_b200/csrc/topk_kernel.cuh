@@ -767,7 +767,7 @@ __device__ __forceinline__ Filter refilter_from_global(Smem& s, Filter f, RowSpa
   return f;
 }
 
-// The need-th largest of the kSampleVals sampled keys in fkey, to within
+// The need-th largest of the nvals sampled keys in fkey, to within
 // one bin of a second histogram round (1 <= need <= the number sampled; every
 // sampled key lies in [lo, hi]). Round one counts 1024 bins over a 10-bit
 // slice of [lo, hi] below its highest differing bit and finds, from the top,
@@ -854,14 +854,6 @@ __device__ __forceinline__ uint32_t sample_kth(Smem& s, int nvals, uint32_t need
   return __reduce_min_sync(kFull, lane < kFilterWarps ? s.fred[3][lane] : 0xFFFFFFFFu);
 }
 
-// A threshold for an item with no estimate, from a sample of kSampleVals
-// values in kSampleChunks evenly spaced runs of 128 (aligned 16-byte blocks
-// inside the item): the value with as many sampled values above it as 1.25
-// times the share of m in the sample, plus 12. On a 128K-value row with k =
-// 2048 that lets about 2.9K values through, some three standard deviations of
-// the sample's count above m: a re-read is rare, and a looser margin costs
-// more in candidate writes and compactions than it saves. Returns -inf when
-// the sample gives none.
 // Loads kFilterWarps * kRunsPerWarp evenly spaced runs of 128 values (aligned
 // 16-byte blocks inside the item) into fkey as keys, 0 for a position outside
 // [0, L) (below every key), and returns their smallest and largest key in
@@ -908,16 +900,27 @@ __device__ __forceinline__ void sample_keys(Smem& s, const T* row, int64_t L, in
 // times the share of m in the sample, plus 12. On a 128K-value row with k =
 // 2048 that lets about 2.9K values through, some three standard deviations of
 // the sample's count above m: a re-read is rare, and a looser margin costs
-// more in candidate writes and compactions than it saves. Returns -inf when
-// the sample gives none.
+// more in candidate writes and compactions than it saves. With `few` (each
+// CTA has at most two rows, so most rows sample) half as many values are
+// sampled: the sample's cost then counts for more than the looser threshold;
+// with many rows per CTA only a CTA's first row samples, and the rows after it
+// start from thresholds carried from it. Returns -inf when the sample gives
+// none.
 template <class T>
-__device__ __noinline__ float sample_threshold(const T* row, int64_t L, int m, int tid) {
+__device__ __noinline__ float sample_threshold(const T* row, int64_t L, int m, int tid, bool few) {
   Smem& s = cta_smem();
   uint32_t mn, mx;
-  sample_keys<T, kSampleRunsPerWarp>(s, row, L, tid, mn, mx);
-  const double share = static_cast<double>(kSampleVals) * m / static_cast<double>(L);
-  const uint32_t need = min(static_cast<uint32_t>(kSampleVals - 8), static_cast<uint32_t>(1.25 * share) + 12u);
-  const uint32_t T0 = sample_kth(s, kSampleVals, need, mn, mx, tid);
+  int nvals;
+  if (few) {
+    sample_keys<T, kSampleRunsPerWarp / 2>(s, row, L, tid, mn, mx);
+    nvals = kSampleVals / 2;
+  } else {
+    sample_keys<T, kSampleRunsPerWarp>(s, row, L, tid, mn, mx);
+    nvals = kSampleVals;
+  }
+  const double share = static_cast<double>(nvals) * m / static_cast<double>(L);
+  const uint32_t need = min(static_cast<uint32_t>(nvals - 8), static_cast<uint32_t>(1.25 * share) + 12u);
+  const uint32_t T0 = sample_kth(s, nvals, need, mn, mx, tid);
   bar_filter();  // fkey, fidx, fred and bc are free again
   return (T0 == 0u || T0 >= kInfKey) ? __int_as_float(0xff800000) : from_key(T0);
 }
@@ -1666,7 +1669,7 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
       }
     }
     if (m == k && !spec && L >= kSampleMinLen) {
-      const float ts = sample_threshold(rowp, L, m, tid);
+      const float ts = sample_threshold(rowp, L, m, tid, p.num_rows <= 2 * static_cast<int64_t>(gridDim.x));
       if (ts > __int_as_float(0xff800000)) {
         spec = true;
         f.t = ts;

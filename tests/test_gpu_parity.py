@@ -356,7 +356,8 @@ def test_few_levels_many_rows(oracle_mod, dsa):
     assert_parity(oracle_mod, dsa, x, L, 100)
 
 
-SAMPLE_RUNS = 32    # a row's first threshold is sampled from 32 runs of 128 values
+SAMPLE_RUNS = 32    # a row's first threshold is sampled from 32 runs of 128 values,
+FEW_ROWS_SAMPLE_RUNS = 16  # or 16 when every CTA has at most two rows
 CLUSTER_SAMPLE_RUNS = 8  # a cluster rank's from 8 (one per filter warp)
 CHUNK_ALIGN = 8     # a cluster rank's chunk is rounded up to a multiple of 8 elements
 
@@ -375,7 +376,7 @@ def test_sampled_threshold_fallback_many_rows(oracle_mod, dsa):
     rng = np.random.default_rng(5)
     rows, L, stride = 148, 120000, 131072  # one row per CTA: every row is a first row
     x = (rng.standard_normal((rows, stride)) * 0.01).astype(np.float32)
-    for b in _sample_runs(L, SAMPLE_RUNS):
+    for b in sorted(set(_sample_runs(L, SAMPLE_RUNS)) | set(_sample_runs(L, FEW_ROWS_SAMPLE_RUNS))):
         x[:, b:b + 128] = 100.0 + rng.random((rows, 128), dtype=np.float32)
     Ls = np.full(rows, L, np.int32)
     dsa.device_status(clear=True)
