@@ -184,11 +184,13 @@ def test_cluster_threshold_shared_by_ranks(oracle_mod, dsa, dtype):
     Rows where it lies far from a rank's own share: values rising along the
     row (the whole top k in the last chunk), 1000 large values placed between
     two sample runs of one chunk, one chunk of shifted values on a coarse grid
-    (ties at the cut), and a plain row of another length."""
+    (ties at the cut), a plain row of another length, a row too short for any
+    rank to sample (no threshold: ranks keep every value above -inf) and an
+    empty row."""
     import torch
     rng = np.random.default_rng(3500 + (dtype == "bf16"))
-    rows, stride, k = 4, 600000, 2048
-    L = np.array([stride, stride - 5, stride, 400001], np.int32)
+    rows, stride, k = 6, 600000, 2048
+    L = np.array([stride, stride - 5, stride, 400001, 20000, 0], np.int32)
     x = rng.standard_normal((rows, stride)).astype(np.float32)
     x[0] = np.sort(x[0])
     x[1, 302000:303000] += 50.0  # inside one rank's chunk, clear of its sample runs
