@@ -132,6 +132,80 @@ def test_cluster_path_many_rows(oracle_mod, dsa):
     assert_parity(oracle_mod, dsa, x, L, 2048)
 
 
+@pytest.mark.parametrize("seed", range(16))
+def test_rows_random_shapes(oracle_mod, dsa, seed):
+    """Seeded random many-row launches: 32-500 rows (one or two per CTA, where
+    first rows sample 2048 values, or more, where they sample 4096 and later
+    rows carry thresholds), strides 1000-200000 (the one-stage instance
+    included), lengths from 0 to the stride, k from 1 to 2048, fp32 or bf16,
+    and per row one of several value patterns."""
+    rng = np.random.default_rng(3900 + seed)
+    rows = int(rng.integers(32, 501))
+    stride = int(rng.integers(1000, 200001))
+    k = (2048, 512, 7, 2048, 1024, 1, 2048, 100)[seed % 8]
+    L = rng.integers(0, stride + 1, size=rows).astype(np.int32)
+    L[rng.random(rows) < 0.3] = stride
+    x = rng.standard_normal((rows, stride)).astype(np.float32)
+    kinds = rng.integers(0, 6, size=rows)
+    x[kinds == 1] = np.round(x[kinds == 1] * 4) / 4
+    x[kinds == 2] = rng.integers(0, 4, (int((kinds == 2).sum()), stride)).astype(np.float32)
+    x[kinds == 3] = np.where(rng.random((int((kinds == 3).sum()), stride)) < 0.01, x[kinds == 3], -np.inf)
+    x[kinds == 4] = np.sort(x[kinds == 4], axis=1)
+    x[kinds == 5] = x[kinds == 5] - 2.0 * np.arange(int((kinds == 5).sum()))[:, None]
+    t = torch.from_numpy(x)
+    if seed % 2:
+        t = t.to(torch.bfloat16)
+    if dsa.plan(rows, stride, k)[0] != 1:
+        pytest.skip("this shape takes clusters on this GPU")
+    dsa.device_status(clear=True)
+    got = dsa.dsa_topk(t.cuda(), torch.from_numpy(L).cuda(), k).cpu().numpy()
+    exp = oracle_mod.topk(t.float().numpy(), L, k)
+    np.testing.assert_array_equal(got, exp)
+    assert dsa.device_status() & dsa.STATUS_ERRORS == 0
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_cluster_random_shapes(oracle_mod, dsa, seed):
+    """Seeded random cluster launches: 1-8 rows, strides 200K-700K, lengths
+    from 0 to the stride, k from 1 to 2048, fp32 or bf16, and per row one of
+    several value patterns (normal, a coarse grid, four levels, mostly -inf,
+    sorted either way, a block of large values), so the shared threshold, the
+    merge's retry and its tie split meet many combinations."""
+    rng = np.random.default_rng(3700 + seed)
+    rows = int(rng.integers(1, 9))
+    stride = int(rng.integers(200000, 700001))
+    k = (2048, 7, 1024, 1, 2048, 512, 2048, 1024)[seed % 8]
+    L = rng.integers(0, stride + 1, size=rows).astype(np.int32)
+    L[rng.random(rows) < 0.3] = stride
+    x = rng.standard_normal((rows, stride)).astype(np.float32)
+    for r in range(rows):
+        kind = int(rng.integers(0, 7))
+        if kind == 1:
+            x[r] = np.round(x[r] * 4) / 4
+        elif kind == 2:
+            x[r] = rng.integers(0, 4, stride).astype(np.float32)
+        elif kind == 3:
+            keep = rng.random(stride) < 0.001
+            x[r] = np.where(keep, x[r], -np.inf)
+        elif kind == 4:
+            x[r] = np.sort(x[r])
+        elif kind == 5:
+            x[r] = np.sort(x[r])[::-1]
+        elif kind == 6:
+            b = int(rng.integers(0, stride - 3000))
+            x[r, b:b + 3000] += 40.0
+    t = torch.from_numpy(x)
+    if seed % 2:
+        t = t.to(torch.bfloat16)
+    if dsa.plan(rows, stride, k)[0] == 1:
+        pytest.skip("this shape takes one CTA per row on this GPU")
+    dsa.device_status(clear=True)
+    got = dsa.dsa_topk(t.cuda(), torch.from_numpy(L).cuda(), k).cpu().numpy()
+    exp = oracle_mod.topk(t.float().numpy(), L, k)
+    np.testing.assert_array_equal(got, exp)
+    assert dsa.device_status() & dsa.STATUS_ERRORS == 0
+
+
 @pytest.mark.parametrize("stride_of_run", [1, 2, 3])
 @pytest.mark.parametrize("shape", ["rows", "cluster"])
 def test_tied_runs_index_cut(oracle_mod, dsa, stride_of_run, shape):
