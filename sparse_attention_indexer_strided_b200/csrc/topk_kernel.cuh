@@ -2016,7 +2016,7 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
       s.bc[3] = any_full ? B : gmin;
       s.bc[4] = gmax;
       s.bc[5] = gmin;
-      s.spub[3] = kdall;  // read by the leader's ranking
+      s.spub[3] = kdall;  // read below and by the leader's ranking
       s.abort_any = any_ab ? 1u : 0u;
       // fewer than m candidates under a guessed threshold: values below it
       // are needed, so every rank takes its chunk again with no threshold
@@ -2038,11 +2038,14 @@ __device__ __noinline__ uint32_t cluster_merge(uint32_t n_r, uint32_t m, bool ab
   }
   uint32_t need = m;
   bool exact = false;
-  // Everything goes to the leader when it fits and holds little more than m;
-  // otherwise at least one round narrows it (with values on a coarse grid,
-  // usually to m plus one tied level: a leader ranking twice m tied
-  // candidates costs more than the round)
-  if (N <= static_cast<uint32_t>(kHandCap) && N <= m + (m >> 3)) {
+  // Everything goes to the leader when it fits, unless the candidates sit on
+  // a coarse value grid (keys differing only from bit 8 up, as bf16 values
+  // do) and number more than m by an eighth: then at least one round narrows
+  // them, usually to m plus one tied level (a leader ranking twice m tied
+  // candidates costs more than the round; off a grid it costs less)
+  const uint32_t kdg = s.spub[3];  // the key-difference bits, the same in every rank
+  const bool coarse = kdg == 0u || __ffs(kdg) - 1 >= 8;
+  if (N <= static_cast<uint32_t>(kHandCap) && (N <= m + (m >> 3) || !coarse)) {
     lo = gmin;
   } else {
     // ---- phase 2: cluster-wide histogram rounds until the survivors fit
