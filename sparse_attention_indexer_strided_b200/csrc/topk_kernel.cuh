@@ -18,10 +18,10 @@
 //                                  cut when one suffices, else an exact select
 //                                  with the tie cut by index. At the end of the
 //                                  row the candidates are handed over.
-//   finisher (6 warps)           : ranks the handed-over candidates by (key
-//                                  descending, index ascending) with bucket
-//                                  passes over a composite key (a bitonic sort
-//                                  when a bucket stays crowded with equal
+//   finisher (6 warps; 7 for     : ranks the handed-over candidates by (key
+//   16-bit logits)                 descending, index ascending) with bucket
+//                                  passes over a composite key (an LSD radix
+//                                  sort when a bucket stays crowded with equal
 //                                  keys), then writes the first m indices and
 //                                  -1 padding while the filter warps already
 //                                  stream the next row.
@@ -63,11 +63,21 @@ namespace rows {
 
 constexpr int kFilterWarps = 8;
 constexpr int kFilterThreads = kFilterWarps * 32;  // 256
-constexpr int kFinishWarps = 6;
-constexpr int kFinishThreads = kFinishWarps * 32;  // 192
-constexpr int kJointThreads = kFilterThreads + kFinishThreads;  // 448: both ranking a CTA's last row
-constexpr int kProducerWarp = kFilterWarps + kFinishWarps;
-constexpr int kThreads = 16 * 32;                       // 512: many-row mode (4 warpgroups; warp 15 idle)
+// Finisher warps of the many-row kernel, by element type. With 16-bit logits
+// the ranking (values tied on a coarse grid, sorted) bounds a row, so it takes
+// the spare warp too; with fp32 the finisher keeps up with six, and a
+// seventh only takes issue slots from the streaming filter warps.
+template <class T>
+__host__ __device__ constexpr int finish_warps() { return sizeof(T) == 4 ? 6 : 7; }
+constexpr int kFinishWarpsMax = 7;
+constexpr int kNredWarps = kFilterWarps + 6;  // warps whose reductions sit in Smem::nred
+template <class T>
+__host__ __device__ constexpr int finish_threads() { return finish_warps<T>() * 32; }  // 192 or 224
+template <class T>
+__host__ __device__ constexpr int joint_threads() { return kFilterThreads + finish_threads<T>(); }  // both ranking a CTA's last row
+template <class T>
+__host__ __device__ constexpr int producer_warp() { return kFilterWarps + finish_warps<T>(); }
+constexpr int kThreads = 16 * 32;                       // 512: many-row mode (filter, finisher, producer warps)
 constexpr int kClusterWarp = kFilterWarps;              // cluster mode: the producer warp
 constexpr int kClusterThreads = 12 * 32;                // 384: cluster mode (3 warpgroups; warps 9-11 only mirror barriers)
 constexpr int kGroups = 8;                              // groups of 4 values per lane and stage
@@ -129,7 +139,7 @@ struct __align__(128) Smem {
   uint32_t hist[256];         // filter radix histogram
   uint4 red[2][(kFilterWarps + 3) / 4];  // per-warp survivor counts, by stage parity
   uint32_t fred[4][kFilterWarps];
-  uint32_t nred[5][kFilterWarps + kFinishWarps];  // finisher per-warp reductions (6, 8 or 14 warps)
+  uint32_t nred[5][kNredWarps];  // finisher per-warp reductions (6 to 14 warps; a 15th: nred_x)
   uint32_t bc[8];
   uint32_t small[32];
   uint32_t rec[2];  // finisher: keys at ranks k-1 and 3k/4-1
@@ -156,6 +166,10 @@ struct __align__(128) Smem {
   uint32_t merge_retry;
   unsigned long long full[kMaxStages], empty[kMaxStages];
   unsigned long long hfull, hempty;
+  // the 15th warp's per-warp reductions (a joint ranking with seven finisher
+  // warps), kept apart so that every other field has the offset it has with
+  // six: the block's layout measurably changes the streaming loop's speed
+  uint32_t nred_x[5];
 };
 static_assert(sizeof(Smem) <= 232448, "shared memory budget of one CTA per SM");
 
@@ -1047,10 +1061,19 @@ struct Finisher {
   static constexpr int kBuckets = kBucketMax / (4 * NT) * (4 * NT);  // 3840, 4096 or 3584
   static constexpr int kScanPer = kBuckets / NT;  // counters per thread
   static_assert(kBuckets <= kBucketMax && kBuckets >= 2048 && kScanPer % 4 == 0 &&
-                    kWarps <= kFilterWarps + kFinishWarps,
+                    kWarps <= kFilterWarps + kFinishWarpsMax,
                 "bucket counters split evenly over the threads; bucket_shift narrows a slice by one bit at most");
 
   __device__ __forceinline__ static void bar() { asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory"); }
+
+  // per-warp reduction slot i of warp w
+  __device__ __forceinline__ static uint32_t& nred(Smem& s, int i, int w) {
+    if constexpr (kWarps > kNredWarps) {
+      return w < kNredWarps ? s.nred[i][w] : s.nred_x[i];
+    } else {
+      return s.nred[i][w];
+    }
+  }
 
   __device__ __forceinline__ static int bucket_shift(uint64_t cmax) {
     const int bits = cmax ? 64 - __clzll(static_cast<long long>(cmax)) : 0;
@@ -1335,10 +1358,10 @@ struct Finisher {
     or_lo = __reduce_or_sync(kFull, or_lo);
     and_lo = __reduce_and_sync(kFull, and_lo);
     if (lane == 0) {
-      s.nred[0][fw] = or_hi;
-      s.nred[1][fw] = and_hi;
-      s.nred[2][fw] = or_lo;
-      s.nred[3][fw] = and_lo;
+      nred(s, 0, fw) = or_hi;
+      nred(s, 1, fw) = and_hi;
+      nred(s, 2, fw) = or_lo;
+      nred(s, 3, fw) = and_lo;
     }
     bar();
     const int ns = static_cast<int>(s.bc[6]);
@@ -1347,10 +1370,10 @@ struct Finisher {
       uint32_t a0 = 0u, a1 = 0xFFFFFFFFu, b0 = 0u, b1 = 0xFFFFFFFFu;
 #pragma unroll
       for (int ww = 0; ww < kWarps; ++ww) {
-        a0 |= s.nred[0][ww];
-        a1 &= s.nred[1][ww];
-        b0 |= s.nred[2][ww];
-        b1 &= s.nred[3][ww];
+        a0 |= nred(s, 0, ww);
+        a1 &= nred(s, 1, ww);
+        b0 |= nred(s, 2, ww);
+        b1 &= nred(s, 3, ww);
       }
       vhi = a0 & ~a1;
       vlo = b0 & ~b1;
@@ -1407,18 +1430,18 @@ struct Finisher {
       imax = __reduce_max_sync(kFull, imax);
       kdiff = __reduce_or_sync(kFull, kdiff);
       if (lane == 0) {
-        s.nred[0][fw] = kmin;
-        s.nred[1][fw] = kmax;
-        s.nred[2][fw] = imax;
-        s.nred[3][fw] = kdiff;
+        nred(s, 0, fw) = kmin;
+        nred(s, 1, fw) = kmax;
+        nred(s, 2, fw) = imax;
+        nred(s, 3, fw) = kdiff;
       }
       bar();
 #pragma unroll
       for (int ww = 0; ww < kWarps; ++ww) {
-        kmin = min(kmin, s.nred[0][ww]);
-        kmax = max(kmax, s.nred[1][ww]);
-        imax = max(imax, s.nred[2][ww]);
-        kdiff |= s.nred[3][ww];
+        kmin = min(kmin, nred(s, 0, ww));
+        kmax = max(kmax, nred(s, 1, ww));
+        imax = max(imax, nred(s, 2, ww));
+        kdiff |= nred(s, 3, ww);
       }
     }
     // every two keys differ by a multiple of 2^grid (keys on a value grid,
@@ -1485,10 +1508,10 @@ struct Finisher {
         const uint32_t t = __shfl_up_sync(kFull, incl, d);
         if (lane >= d) incl += t;
       }
-      if (lane == 31) s.nred[3][fw] = incl;
+      if (lane == 31) nred(s, 3, fw) = incl;
       bar();
       uint32_t run = incl - sum;
-      for (int ww = 0; ww < fw; ++ww) run += s.nred[3][ww];
+      for (int ww = 0; ww < fw; ++ww) run += nred(s, 3, ww);
       const uint32_t run0 = run;
 #pragma unroll
       for (int i = 0; i < kScanPer / 4; ++i) {
@@ -1517,10 +1540,10 @@ struct Finisher {
       for (int i = 0; i < kScanPer; ++i)
         if (static_cast<uint32_t>(fid * kScanPer + i) <= bm) big = max(big, c[i]);
       big = __reduce_max_sync(kFull, big);
-      if (lane == 0) s.nred[4][fw] = big;
+      if (lane == 0) nred(s, 4, fw) = big;
       bar();
 #pragma unroll
-      for (int ww = 0; ww < kWarps; ++ww) big = max(big, s.nred[4][ww]);
+      for (int ww = 0; ww < kWarps; ++ww) big = max(big, nred(s, 4, ww));
       // a bucket still crowded past the counting limit after a second, finer
       // pass holds values on a coarse grid (equal keys), which finer slices of
       // the same composite range do not split: sort instead (the first pass
@@ -1611,25 +1634,29 @@ struct Finisher {
   }
 };
 
-using RowFinisher = Finisher<kFinishThreads, 2>;
+template <class T>
+using RowFinisher = Finisher<finish_threads<T>(), 2>;
 // the filter warps' own ranking of a cluster leader's row
 using LeaderFinisher = Finisher<kFilterThreads, 1>;
 // a CTA's last row, ranked by the filter and finisher warps together
-using JointFinisher = Finisher<kJointThreads, 3, true>;
+template <class T>
+using JointFinisher = Finisher<joint_threads<T>(), 3, true>;
 
 // Where the filter and finisher warps meet after their row loops. Both roles reach it on every path (a wait that gave up ends a
 // loop early; no loop ends without passing here), so the hardware barrier
 // always completes, and the flag the filter warps wrote before it (s.joint)
 // decides for both whether they rank the row together.
+template <class T>
 __device__ __forceinline__ void joint_rendezvous() {
-  asm volatile("bar.sync 3, %0;" ::"n"(kJointThreads) : "memory");
+  asm volatile("bar.sync 3, %0;" ::"n"(joint_threads<T>()) : "memory");
 }
 
 // The joint ranking, out of line (inlined into the row loops, its registers
 // would be allocated with theirs).
+template <class T>
 __device__ __noinline__ void joint_finish(const Params p, int tid) {
   Smem& s = cta_smem();
-  JointFinisher::finish(s, s.h_n, s.h_m, p.k, s.h_row, p, tid, true);
+  JointFinisher<T>::finish(s, s.h_n, s.h_m, p.k, s.h_row, p, tid, true);
 }
 
 
@@ -1737,8 +1764,8 @@ __device__ void filter_loop(Smem& s, const Params& p, int tid) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.hfull);
   }
-  joint_rendezvous();
-  if (s.joint) joint_finish(p, tid);
+  joint_rendezvous<T>();
+  if (s.joint) joint_finish<T>(p, tid);
 }
 
 
@@ -1764,10 +1791,10 @@ __device__ void finish_loop(Smem& s, const Params& p, int fid) {
   // alone or with these warps)
   for (int64_t row = blockIdx.x; row + gridDim.x < p.num_rows; row += gridDim.x, ++h) {
     const bool ok = mbar_wait_sleep(&s.hfull, h & 1, &s.wait);
-    if (bar_any<2, kFinishThreads>(!ok)) break;  // the filter warps left: nothing more comes
+    if (bar_any<2, finish_threads<T>()>(!ok)) break;  // the filter warps left: nothing more comes
     const int n = s.h_n, m = s.h_m;
     const int64_t L = s.h_len;
-    RowFinisher::finish(s, n, m, k, s.h_row, p, fid, false);
+    RowFinisher<T>::finish(s, n, m, k, s.h_row, p, fid, false);
     if (fid == 0) {
       bool est_ok = false;
       float e = 0.f;
@@ -1781,12 +1808,12 @@ __device__ void finish_loop(Smem& s, const Params& p, int fid) {
       s.est_len[h & 1] = L;
       s.est_ok[h & 1] = est_ok ? 1 : 0;
     }
-    RowFinisher::bar();  // every read of the handover is done, the estimate written
+    RowFinisher<T>::bar();  // every read of the handover is done, the estimate written
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.hempty);
   }
-  joint_rendezvous();
-  if (s.joint) joint_finish(p, kFilterThreads + fid);
+  joint_rendezvous<T>();
+  if (s.joint) joint_finish<T>(p, kFilterThreads + fid);
 }
 
 // ---------------------------------------------------------- producer
@@ -2258,13 +2285,13 @@ __device__ __forceinline__ void cluster_filter(Smem& s, const Params& p, int tid
 }
 
 // Shared state of a fresh CTA (thread 0; a barrier follows).
-__device__ __forceinline__ void init_cta(Smem& s) {
+__device__ __forceinline__ void init_cta(Smem& s, int finish_warps) {
   for (int i = 0; i < kMaxStages; ++i) {
     mbar_init(&s.full[i], 1);
     mbar_init(&s.empty[i], kFilterWarps);
   }
   mbar_init(&s.hfull, kFilterWarps);
-  mbar_init(&s.hempty, kFinishWarps);
+  mbar_init(&s.hempty, finish_warps);
   for (int i = 0; i < 2; ++i) {
     s.est_ok[i] = 0;
     s.est[i] = 0.f;
@@ -2293,14 +2320,14 @@ __global__ void __launch_bounds__(rows::kThreads) topk_rows_kernel(const rows::P
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   rows::Smem& s = *reinterpret_cast<rows::Smem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) rows::init_cta(s);
+  if (tid == 0) rows::init_cta(s, rows::finish_warps<T>());
   __syncthreads();
   pdl_enter();  // every thread: inputs and outputs are touched only after this
   if (warp < rows::kFilterWarps) {
     rows::filter_loop<T, kShort>(s, p, tid);
-  } else if (warp < rows::kProducerWarp) {
+  } else if (warp < rows::producer_warp<T>()) {
     rows::finish_loop<T>(s, p, tid - rows::kFilterThreads);
-  } else if (warp == rows::kProducerWarp && lane == 0) {
+  } else if (warp == rows::producer_warp<T>() && lane == 0) {
     rows::produce_loop<T>(s, p);
   }
 }
@@ -2311,7 +2338,7 @@ __global__ void __launch_bounds__(rows::kThreads) topk_cluster_kernel(const rows
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   rows::Smem& s = *reinterpret_cast<rows::Smem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5;
-  if (tid == 0) rows::init_cta(s);
+  if (tid == 0) rows::init_cta(s, 1);  // no finisher warps: the handover barrier is unused
   __syncthreads();
   pdl_enter();  // every thread: inputs and outputs are touched only after this
   if (warp < rows::kFilterWarps)
